@@ -1,0 +1,363 @@
+"""Throughput of block-causal linear attention (prefill) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl blin|reference] [--config 480p]
+
+One step = one blin_prefill of the whole workload (RoPE table, partial states,
+block scan, output) on inputs already resident in HBM.  The workload defaults
+to the 480p-like latent video: B=1, H=70, d=32, 21 x 30 x 52 tokens, blocks of
+3 frames, bf16 storage.  Inputs (587 MB moved per step) are larger than L2, so
+no flush is needed between steps.  With N > 1 GPUs every rank runs its own
+independent copy of the workload (weak scaling; heads/videos never exchange
+data) and the step time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle (the only reference this
+method has) on a bounded sample of the same workload and prints the same line
+with ``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "block-causal linear-attn tokens·heads/s and % of B200 HBM peak, 1 GPU"
+UNIT = "tokens*heads/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- helpers
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_causal_linear_rope_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches these sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            doc = json.load(f)
+    except Exception:
+        return None
+    if doc.get("source_hash") != kernel_source_hash():
+        return None
+    return doc.get("per_launch_bytes", {}).get(workload, {}).get(kernel)
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(ngpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample(w: workloads.Workload, q, k, v, rows_total: int, seed: int = 0):
+    """Time the explicit pair-sum oracle on `rows_total` seeded query rows (all heads)."""
+    import oracle
+    pos, blk = oracle.grid(w.T, w.Hg, w.Wg, w.F)
+    rows = np.sort(np.random.default_rng([seed, 5]).choice(w.N, size=rows_total, replace=False))
+    qs = q.reshape(-1, w.N, w.d)
+    ks = k.reshape(-1, w.N, w.d)
+    vs = v.reshape(-1, w.N, w.d)
+    t0 = time.perf_counter()
+    oracle.attention_rows(qs, ks, vs, pos, blk, rows, w.split, w.theta, w.eps)
+    dt = time.perf_counter() - t0
+    return rows_total * qs.shape[0] / dt, dt
+
+
+def omp_threads() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    q, k, v = workloads.call_tensors(w)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, rows, seed=1)
+    times = []
+    for i in range(args.steps):
+        _, dt = oracle_sample(w, q, k, v, rows, seed=100 + i)
+        times.append(dt)
+    per_step = sum(times) / len(times)
+    value = rows * w.B * w.H / per_step
+    sample = (f"{rows} seeded query rows x {w.B * w.H} heads of the {w.name} workload per step, "
+              f"explicit O(N^2) float64 pair sum (all keys each row may see)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, world):
+    return {"workload": f"{w.name} prefill: B={w.B} H={w.H} d={w.d} {w.dtype}, latent {w.T}x{w.Hg}x{w.Wg} "
+                        f"(N={w.N}), blocks of {w.F} frames, RoPE split {w.split}, theta {w.theta:g}, eps {w.eps:g}",
+            "tokens_per_head": w.N, "heads_per_gpu": w.B * w.H, "head_dim": w.d, "block_frames": w.F,
+            "l2": "inputs larger than L2 (no flush)", "parallelism": f"independent replica per GPU x{world}"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_blin(args, w):
+    import torch
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    import block_causal_linear_rope_b200 as blin
+
+    dt_t = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    wr = w.with_(seed=w.seed + rank)
+    q, k, v = workloads.call_tensors(wr)
+    qh, kh, vh = (torch.from_numpy(x).to(dt_t).pin_memory() for x in (q, k, v))
+    qd, kd, vd = (x.to("cuda") for x in (qh, kh, vh))
+    od = torch.empty_like(qd)
+    oh = torch.empty_like(qh).pin_memory()
+    grid = (w.T, w.Hg, w.Wg)
+    ws = torch.empty(blin.workspace_size(w.B, w.H, w.d, grid, w.F, w.split, w.theta, w.eps),
+                     dtype=torch.uint8, device="cuda")
+
+    # pre-marshalled C-ABI arguments: the timed loop calls blin_prefill directly
+    geom = blin._geom(w.T, w.Hg, w.Wg, w.F, w.split, w.theta, w.eps)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    cargs = (ctypes.c_void_p(qd.data_ptr()), ctypes.c_void_p(kd.data_ptr()), ctypes.c_void_p(vd.data_ptr()),
+             ctypes.c_void_p(od.data_ptr()), blin.BF16 if w.dtype == "bf16" else blin.F32, w.B, w.H, w.d,
+             ctypes.byref(geom), None, ctypes.c_void_p(ws.data_ptr()), ws.numel(), stream)
+    prefill_c = blin.lib.blin_prefill
+
+    def step():
+        rc = prefill_c(*cargs)
+        if rc != 0:
+            raise RuntimeError(blin.lib.blin_last_error().decode())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+
+    timer = blin.LaunchTimer()
+    sets = [timer.new_set() for _ in range(args.steps)]
+    arm = blin.LaunchTimer.arm_set
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)  # let the sampler start
+        start.record()
+        for i in range(args.steps):
+            arm(sets[i])
+            step()
+        end.record()
+        torch.cuda.synchronize()
+        blin.lib.blin_set_timing_events(None, 0)
+        time.sleep(0.25)
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms, world)
+    per_kernel = timer.elapsed_ms()
+    avg = {kname: sum(d[kname] for d in per_kernel) / len(per_kernel) for kname in blin.KERNELS}
+    status = blin.device_status()
+    if status != 0:
+        raise SystemExit(f"kernel watchdog fired (code {status})")
+
+    # ---- end to end through the C ABI: pinned host inputs in, host output back
+    h2d = 3 * qh.numel() * qh.element_size()
+    d2h = oh.numel() * oh.element_size()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(od, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, args.steps // 4)
+    e_start.record()
+    for _ in range(e_steps):
+        e2e_step()
+    e_end.record()
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e_start.elapsed_time(e_end) / e_steps, world)
+
+    units = w.B * w.H * w.N  # token*heads per GPU per step
+    value = units * world / (ms * 1e-3)
+    e2e_value = units * world / (e_ms * 1e-3)
+
+    # ---- roofline of the dominant kernel (algorithmic bytes / live event time)
+    elem = 2 if w.dtype == "bf16" else 4
+    alg = {"partial_states": 2 * units * w.d * elem,  # K and V read
+           "output": 2 * units * w.d * elem}          # Q read, O written
+    dom = max(("partial_states", "output"), key=lambda k_: avg[k_])
+    peak, peak_kind = hbm_peak()
+    achieved = alg[dom] / (avg[dom] * 1e-3) / 1e9
+    whole = 4 * units * w.d * elem / (ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": config_dict(w, world),
+        "hbm_gbs_whole_step": whole, "hbm_frac_whole_step": whole / peak,
+        "kernel_ms": avg,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": recorded_traffic(dom, w.name),
+                     "algorithmic_bytes_per_launch": alg[dom]},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, secs = oracle_sample(w, q, k, v, args.cpu_rows)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+                                "sample": f"{args.cpu_rows} seeded query rows x {w.B * w.H} heads of {w.name}, "
+                                          f"explicit O(N^2) float64 pair sum, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="blin", choices=["blin", "reference"])
+    ap.add_argument("--config", default="480p", choices=["480p", "720p", "wide"])
+    ap.add_argument("--cpu-rows", type=int, default=96, help="oracle rows for the CPU baseline")
+    ap.add_argument("--ref-rows", type=int, default=24, help="oracle rows per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = workloads.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_blin(args, w)
+
+
+if __name__ == "__main__":
+    main()

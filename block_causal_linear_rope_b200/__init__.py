@@ -1,0 +1,290 @@
+"""Block-causal ReLU linear attention with numerator-only 3D RoPE on B200.
+
+Python binding of ``libblin.so`` (C ABI declared in ``include/blin.h``).  This
+module only marshals arguments: every step of the computation runs in the
+library's CUDA kernels.  PyTorch supplies device memory and the current stream.
+
+    import block_causal_linear_rope_b200 as blin
+    o = blin.prefill(q, k, v, grid=(T, Hg, Wg), block_frames=3, rope_split=(8, 12, 12))
+    st = blin.BlockState(B, H, d)
+    o_b = blin.block_step(q_b, k_b, v_b, Hg, Wg, frames=3, rope_split=(8, 12, 12), state=st)
+
+Tensors are contiguous [B, H, N, d] (d = 32 or 64) in float32 or bfloat16 on
+the current CUDA device.  If the library is missing this import raises: there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = ["BlinError", "BlockState", "prefill", "block_step", "workspace_size", "device_status",
+           "LaunchTimer", "KERNELS", "lib", "LIB_PATH", "F32", "BF16"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libblin.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "BLIN_OK", -1: "BLIN_ERR_INVALID_ARG", -2: "BLIN_ERR_SHAPE", -3: "BLIN_ERR_DTYPE",
+           -4: "BLIN_ERR_ALIGN", -5: "BLIN_ERR_WORKSPACE", -6: "BLIN_ERR_STATE", -7: "BLIN_ERR_CUDA",
+           -8: "BLIN_ERR_DEVICE"}
+
+
+class BlinError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Geom(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("Hgt", ctypes.c_int), ("Wid", ctypes.c_int),
+                ("block_frames", ctypes.c_int), ("rope_split", ctypes.c_int * 3),
+                ("theta", ctypes.c_float), ("eps", ctypes.c_float)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python block_causal_linear_rope_b200/build.py` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    L.blin_state_init.argtypes = [I, I, I, P, ctypes.POINTER(P)]
+    L.blin_state_free.argtypes = [P]
+    L.blin_state_reset.argtypes = [P, P]
+    L.blin_state_tensors.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(I)]
+    L.blin_state_bytes.argtypes = [P]
+    L.blin_state_bytes.restype = S
+    L.blin_state_copy_to_host.argtypes = [P, P, S, P]
+    L.blin_state_copy_from_host.argtypes = [P, P, S, I, P]
+    L.blin_state_reserve.argtypes = [P, ctypes.c_long, P]
+    L.blin_prefill_workspace_size.argtypes = [I, I, I, ctypes.POINTER(Geom)]
+    L.blin_prefill_workspace_size.restype = S
+    L.blin_prefill.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), P, P, S, P]
+    L.blin_block_step.argtypes = [P, P, P, P, I, I, I, I, I, I, I, ctypes.POINTER(I * 3), F, F, P, I, P]
+    L.blin_last_error.restype = ctypes.c_char_p
+    L.blin_device_status.argtypes = [ctypes.POINTER(I)]
+    L.blin_version.restype = ctypes.c_char_p
+    L.blin_set_timing_events.argtypes = [P, I]
+    L.blin_set_timing_events.restype = I
+    for fn in ("blin_state_init", "blin_state_free", "blin_state_reset", "blin_state_tensors",
+               "blin_state_copy_to_host", "blin_state_copy_from_host", "blin_state_reserve",
+               "blin_prefill", "blin_block_step", "blin_device_status"):
+        getattr(L, fn).restype = I
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise BlinError(status, lib.blin_last_error().decode())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _geom(T, Hg, Wg, block_frames, rope_split, theta, eps) -> Geom:
+    g = Geom()
+    g.T, g.Hgt, g.Wid, g.block_frames = int(T), int(Hg), int(Wg), int(block_frames)
+    g.rope_split[:] = [int(x) for x in rope_split]
+    g.theta, g.eps = float(theta), float(eps)
+    return g
+
+
+class BlockState:
+    """Constant-size (S, z) cache: S [B,H,d,d], z [B,H,d] fp32 on one device."""
+
+    def __init__(self, B: int, H: int, d: int, stream=None):
+        self.B, self.H, self.d = B, H, d
+        h = ctypes.c_void_p()
+        _check(lib.blin_state_init(B, H, d, _stream(stream), ctypes.byref(h)))
+        self._h = h
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise BlinError(-6, "state already freed")
+        return self._h
+
+    def free(self) -> None:
+        if self._h is not None:
+            _check(lib.blin_state_free(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            if getattr(self, "_h", None) is not None:
+                lib.blin_state_free(self._h)
+        except Exception:
+            pass
+
+    @property
+    def t_next(self) -> int:
+        t = ctypes.c_int()
+        _check(lib.blin_state_tensors(self.handle, None, None, ctypes.byref(t)))
+        return t.value
+
+    @property
+    def nbytes(self) -> int:
+        return int(lib.blin_state_bytes(self.handle))
+
+    def reset(self, stream=None) -> None:
+        _check(lib.blin_state_reset(self.handle, _stream(stream)))
+
+    def reserve(self, max_block_tokens: int, stream=None) -> None:
+        _check(lib.blin_state_reserve(self.handle, int(max_block_tokens), _stream(stream)))
+
+    def to_host(self, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Copy (S, z) into new pinned host tensors (synchronises the stream)."""
+        buf = torch.empty(self.nbytes // 4, dtype=torch.float32, pin_memory=True)
+        s = stream or torch.cuda.current_stream()
+        _check(lib.blin_state_copy_to_host(self.handle, ctypes.c_void_p(buf.data_ptr()), self.nbytes,
+                                           _stream(s)))
+        s.synchronize()
+        n = self.B * self.H * self.d * self.d
+        return (buf[:n].view(self.B, self.H, self.d, self.d).clone(),
+                buf[n:].view(self.B, self.H, self.d).clone())
+
+    def from_host(self, S: torch.Tensor, z: torch.Tensor, t_next: int, stream=None) -> None:
+        """Restore (S, z) and t_next from host tensors (checkpoint resume)."""
+        buf = torch.cat([S.reshape(-1), z.reshape(-1)]).to(torch.float32).contiguous().pin_memory()
+        s = stream or torch.cuda.current_stream()
+        _check(lib.blin_state_copy_from_host(self.handle, ctypes.c_void_p(buf.data_ptr()),
+                                             buf.numel() * 4, int(t_next), _stream(s)))
+        s.synchronize()
+
+
+def _check_qkv(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
+    if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k and v must share shape and dtype")
+
+
+def workspace_size(B: int, H: int, d: int, grid: Sequence[int], block_frames: int,
+                   rope_split: Sequence[int], theta: float = 1e4, eps: float = 1e-6) -> int:
+    g = _geom(*grid, block_frames, rope_split, theta, eps)
+    n = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
+    if n == 0:
+        raise ValueError("invalid shape for blin_prefill")
+    return n
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Sequence[int], block_frames: int,
+            rope_split: Sequence[int], theta: float = 1e4, eps: float = 1e-6,
+            state: Optional[BlockState] = None, out: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Block-causal linear attention over the frames grid=(T, Hg, Wg) (N = T*Hg*Wg)."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    T, Hg, Wg = (int(x) for x in grid)
+    if N != T * Hg * Wg:
+        raise ValueError(f"N={N} but T*Hg*Wg={T * Hg * Wg}")
+    g = _geom(T, Hg, Wg, block_frames, rope_split, theta, eps)
+    if out is None:
+        out = torch.empty_like(q)
+    need = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check(lib.blin_prefill(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                            _dtype_code(q), B, H, d, ctypes.byref(g),
+                            state.handle if state is not None else None,
+                            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)))
+    return out
+
+
+def block_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Hg: int, Wg: int, frames: int,
+               rope_split: Sequence[int], state: BlockState, theta: float = 1e4, eps: float = 1e-6,
+               commit: bool = True, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One autoregressive block of `frames` latent frames read against (and, if
+    commit, added to) the cached state."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    if N != frames * Hg * Wg:
+        raise ValueError(f"N={N} but frames*Hg*Wg={frames * Hg * Wg}")
+    if out is None:
+        out = torch.empty_like(q)
+    split = (ctypes.c_int * 3)(*[int(x) for x in rope_split])
+    _check(lib.blin_block_step(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                               ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                               _dtype_code(q), B, H, d, int(Hg), int(Wg), int(frames),
+                               ctypes.byref(split), float(theta), float(eps), state.handle,
+                               1 if commit else 0, _stream(stream)))
+    return out
+
+
+KERNELS = ("rope_table", "partial_states", "block_scan", "output")
+
+
+class LaunchTimer:
+    """Records CUDA events around each of the library's launches (profiling aid).
+
+    Use ``with LaunchTimer() as t: ...`` around calls on the current thread, then
+    ``t.elapsed_ms()`` (after synchronising) for per-kernel times of the last
+    call.  ``arm()`` re-arms a fresh set of events for the next call.
+    """
+
+    def __init__(self):
+        self.sets = []
+
+    def new_set(self):
+        """Create (and keep) one set of 8 events; returns the C array to arm with."""
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+        for e in evs:  # force creation of the underlying cudaEvent_t
+            e.record()
+        torch.cuda.current_stream().synchronize()
+        arr = (ctypes.c_void_p * 8)(*[e.cuda_event for e in evs])
+        self.sets.append((evs, arr))
+        return arr
+
+    @staticmethod
+    def arm_set(arr) -> None:
+        _check(lib.blin_set_timing_events(ctypes.cast(arr, ctypes.c_void_p), 8))
+
+    def arm(self):
+        arr = self.new_set()
+        self.arm_set(arr)
+        return self.sets[-1][0]
+
+    def __enter__(self):
+        self.arm()
+        return self
+
+    def __exit__(self, *exc):
+        lib.blin_set_timing_events(None, 0)
+        return False
+
+    def elapsed_ms(self):
+        """[{kernel name: ms}] for every armed call (events must have completed)."""
+        out = []
+        for evs, _ in self.sets:
+            out.append({k: evs[2 * i].elapsed_time(evs[2 * i + 1]) for i, k in enumerate(KERNELS)})
+        return out
+
+
+def device_status() -> int:
+    """Synchronise, then read and clear the kernels' watchdog word (0 = clean)."""
+    code = ctypes.c_int(0)
+    rc = lib.blin_device_status(ctypes.byref(code))
+    if rc not in (0, -8):
+        _check(rc)
+    return code.value

@@ -1,0 +1,432 @@
+// Host side of libblin: argument checks, the (S, z) state object, workspace
+// layout, TMA descriptors and the launch sequence of each call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/blin.h"
+#include "blin_internal.cuh"
+
+using namespace blin;
+
+static constexpr uint64_t kStateMagic = 0x626c696e53544154ull;  // "blinSTAT"
+static constexpr uint64_t kFreedMagic = 0xdeadbeefdeadbeefull;
+
+struct blin_state {
+    uint64_t magic;
+    int B, H, d, device;
+    float *S;  // [B][H][d][d]
+    float *z;  // [B][H][d]
+    int t_next;
+    void *scratch;  // block-step workspace (tables, partials, prefix)
+    size_t scratch_bytes;
+};
+
+static thread_local char g_err[512] = "";
+
+static blin_status fail(blin_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+static blin_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(BLIN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- geometry
+struct Plan {
+    KGeom g;
+    int d;
+    size_t tab_bytes, part_bytes, prefix_bytes;
+};
+
+static blin_status check_common(int B, int H, int d, int T, int Hg, int Wg, const int split[3],
+                                float theta, float eps) {
+    if (B < 1 || H < 1) return fail(BLIN_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
+    if (d != 32 && d != 64) return fail(BLIN_ERR_SHAPE, "head dim d must be 32 or 64 (got %d)", d);
+    if (T < 0) return fail(BLIN_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+    if (Hg < 1 || Wg < 1) return fail(BLIN_ERR_INVALID_ARG, "Hgt and Wid must be >= 1 (got %d, %d)", Hg, Wg);
+    if (split == nullptr) return fail(BLIN_ERR_INVALID_ARG, "rope_split is NULL");
+    for (int a = 0; a < 3; ++a)
+        if (split[a] < 0 || (split[a] & 1))
+            return fail(BLIN_ERR_SHAPE, "rope_split entries must be even and >= 0 (got %d,%d,%d)",
+                        split[0], split[1], split[2]);
+    if (split[0] + split[1] + split[2] != d)
+        return fail(BLIN_ERR_SHAPE, "rope_split (%d,%d,%d) must sum to d=%d", split[0], split[1], split[2], d);
+    if (!(theta > 0.f) || !std::isfinite(theta)) return fail(BLIN_ERR_INVALID_ARG, "theta must be finite and > 0");
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(BLIN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const long long HW = (long long)Hg * Wg;
+    const long long N = (long long)T * HW;
+    const long long rows = (long long)B * H * N;
+    if (HW > (1 << 30) || rows >= (1LL << 31) || rows * d >= (1LL << 40))
+        return fail(BLIN_ERR_SHAPE, "problem too large (B*H*N = %lld rows)", rows);
+    return BLIN_OK;
+}
+
+// Builds the call geometry; `one_block` treats the whole call as one block.
+static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0, bool one_block,
+                      const int split[3], float eps, bool for_size = false) {
+    Plan p{};
+    KGeom &g = p.g;
+    p.d = d;
+    g.BH = B * H;
+    g.T = T;
+    g.Hg = Hg;
+    g.Wg = Wg;
+    g.HW = Hg * Wg;
+    g.N = T * g.HW;
+    g.t0 = t0;
+    if (one_block) {
+        g.F = T > 0 ? T : 1;
+        g.first_end = T;
+        g.nblk = T > 0 ? 1 : 0;
+    } else {
+        g.F = F;
+        const int fe = (t0 / F + 1) * F - t0;  // relative frame where the first block ends
+        g.first_end = fe < T ? fe : T;
+        g.nblk = T > 0 ? 1 + (T - g.first_end + F - 1) / F : 0;
+        if (for_size) g.nblk = (T + F - 1) / F + 1;  // worst case over t0
+    }
+    const long long max_blk_tok = (long long)(one_block ? T : (F < T ? F : T)) * g.HW;
+    g.cpb = (int)((max_blk_tok + kChunk - 1) / kChunk);
+    if (g.cpb < 1) g.cpb = 1;
+    const int qtok = kQTiles * kTile;
+    g.qcpb = (int)((max_blk_tok + qtok - 1) / qtok);
+    if (g.qcpb < 1) g.qcpb = 1;
+    g.pt = split[0] / 2;
+    g.py = split[1] / 2;
+    g.px = split[2] / 2;
+    g.eps = eps;
+    g.tab_y = T * g.pt;
+    g.tab_x = g.tab_y + Hg * g.py;
+    const size_t E = (size_t)d * d + d;
+    p.tab_bytes = align256(sizeof(float2) * ((size_t)T * g.pt + (size_t)Hg * g.py + (size_t)Wg * g.px + 1));
+    p.part_bytes = align256(sizeof(float) * (size_t)g.BH * g.nblk * g.cpb * E);
+    p.prefix_bytes = align256(sizeof(float) * (size_t)g.BH * g.nblk * E);
+    return p;
+}
+
+static size_t plan_bytes(const Plan &p) { return 256 + p.tab_bytes + p.part_bytes + p.prefix_bytes; }
+
+static void plan_bind(Plan &p, void *ws) {
+    uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255);
+    p.g.tab = reinterpret_cast<const float2 *>(base);
+    p.g.part = reinterpret_cast<float *>(base + p.tab_bytes);
+    p.g.prefix = reinterpret_cast<float *>(base + p.tab_bytes + p.part_bytes);
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2D map over [rows][d] bf16 rows, 128-row boxes, swizzle = row width (64 B / 128 B).
+static bool make_map(CUtensorMap *m, const void *base, long long rows, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)kTile};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launch sequence
+static thread_local cudaEvent_t const *g_timing = nullptr;
+
+static void mark(int i, bool after, cudaStream_t s) {
+    if (g_timing != nullptr) cudaEventRecord(g_timing[2 * i + (after ? 1 : 0)], s);
+}
+
+static blin_status run(Plan &p, const void *q, const void *k, const void *v, void *o, blin_dtype dt,
+                       const float *S_in, const float *z_in, float *S_out, float *z_out, double theta,
+                       const int split[3], cudaStream_t s) {
+    const KGeom &g = p.g;
+    const int d = p.d;
+    const bool tc = dt == BLIN_BF16 && tc_supported(d, split);
+    CUtensorMap mq, mk, mv, mo;
+    if (tc) {
+        const long long rows = (long long)g.BH * g.N;
+        if (!make_map(&mq, q, rows, d) || !make_map(&mk, k, rows, d) || !make_map(&mv, v, rows, d) ||
+            !make_map(&mo, o, rows, d))
+            return fail(BLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
+    }
+    const bool bf = dt == BLIN_BF16;
+    cudaError_t e;
+    mark(0, false, s);
+    if ((e = launch_rope_table(g, theta, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
+    mark(0, true, s);
+    mark(1, false, s);
+    e = tc ? launch_partial_tc(g, d, mk, mv, s) : launch_partial_simt(g, d, bf, k, v, s);
+    if (e != cudaSuccess) return cuda_fail(e, "partial-state launch");
+    mark(1, true, s);
+    mark(2, false, s);
+    if ((e = launch_scan(g, d, S_in, z_in, S_out, z_out, s)) != cudaSuccess) return cuda_fail(e, "scan launch");
+    mark(2, true, s);
+    mark(3, false, s);
+    e = tc ? launch_output_tc(g, d, mq, mo, o, s) : launch_output_simt(g, d, bf, q, o, s);
+    if (e != cudaSuccess) return cuda_fail(e, "output launch");
+    mark(3, true, s);
+    return BLIN_OK;
+}
+
+static blin_status check_state(const blin_state *st) {
+    if (st == nullptr) return fail(BLIN_ERR_INVALID_ARG, "state is NULL");
+    if (st->magic != kStateMagic) return fail(BLIN_ERR_STATE, "state handle is not live (freed or foreign)");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != st->device)
+        return fail(BLIN_ERR_STATE, "state lives on device %d but the current device is %d", st->device, dev);
+    return BLIN_OK;
+}
+
+static blin_status check_io(const void *q, const void *k, const void *v, void *o, blin_dtype dt) {
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
+        return fail(BLIN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL device pointers");
+    if (dt != BLIN_F32 && dt != BLIN_BF16) return fail(BLIN_ERR_DTYPE, "unknown dtype %d", (int)dt);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(BLIN_ERR_ALIGN, "q, k, v and o must be 16-byte aligned");
+    return BLIN_OK;
+}
+
+extern "C" {
+
+const char *blin_last_error(void) { return g_err; }
+
+const char *blin_version(void) { return "blin 0.1 (sm_100a)"; }
+
+blin_status blin_state_init(int B, int H, int d, blin_stream stream, blin_state **out) {
+    if (out == nullptr) return fail(BLIN_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (B < 1 || H < 1) return fail(BLIN_ERR_INVALID_ARG, "B and H must be >= 1");
+    if (d != 32 && d != 64) return fail(BLIN_ERR_SHAPE, "d must be 32 or 64");
+    blin_state *st = new blin_state{};
+    st->magic = kStateMagic;
+    st->B = B;
+    st->H = H;
+    st->d = d;
+    cudaError_t e = cudaGetDevice(&st->device);
+    const size_t sb = sizeof(float) * (size_t)B * H * d * d, zb = sizeof(float) * (size_t)B * H * d;
+    if (e == cudaSuccess) e = cudaMalloc(&st->S, sb);
+    if (e == cudaSuccess) e = cudaMalloc(&st->z, zb);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(st->S, 0, sb, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(st->z, 0, zb, s);
+    if (e != cudaSuccess) {
+        if (st->S) cudaFree(st->S);
+        if (st->z) cudaFree(st->z);
+        delete st;
+        return cuda_fail(e, "state allocation");
+    }
+    *out = st;
+    return BLIN_OK;
+}
+
+blin_status blin_state_free(blin_state *st) {
+    if (st == nullptr) return BLIN_OK;
+    if (st->magic != kStateMagic) return fail(BLIN_ERR_STATE, "state handle is not live (double free?)");
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(st->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    cudaFree(st->S);
+    cudaFree(st->z);
+    if (st->scratch) cudaFree(st->scratch);
+    cudaSetDevice(prev);
+    st->magic = kFreedMagic;
+    delete st;
+    if (e != cudaSuccess) return cuda_fail(e, "synchronise before state free");
+    return BLIN_OK;
+}
+
+blin_status blin_state_reset(blin_state *st, blin_stream stream) {
+    blin_status rc = check_state(st);
+    if (rc != BLIN_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t sb = sizeof(float) * (size_t)st->B * st->H * st->d * st->d;
+    const size_t zb = sizeof(float) * (size_t)st->B * st->H * st->d;
+    cudaError_t e = cudaMemsetAsync(st->S, 0, sb, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(st->z, 0, zb, s);
+    if (e != cudaSuccess) return cuda_fail(e, "state reset");
+    st->t_next = 0;
+    return BLIN_OK;
+}
+
+blin_status blin_state_tensors(const blin_state *st, float **S, float **z, int *t_next) {
+    if (st == nullptr) return fail(BLIN_ERR_INVALID_ARG, "state is NULL");
+    if (st->magic != kStateMagic) return fail(BLIN_ERR_STATE, "state handle is not live");
+    if (S) *S = st->S;
+    if (z) *z = st->z;
+    if (t_next) *t_next = st->t_next;
+    return BLIN_OK;
+}
+
+size_t blin_state_bytes(const blin_state *st) {
+    if (st == nullptr || st->magic != kStateMagic) return 0;
+    return sizeof(float) * (size_t)st->B * st->H * ((size_t)st->d * st->d + st->d);
+}
+
+blin_status blin_state_copy_to_host(const blin_state *st, void *host, size_t bytes, blin_stream stream) {
+    blin_status rc = check_state(st);
+    if (rc != BLIN_OK) return rc;
+    if (host == nullptr) return fail(BLIN_ERR_INVALID_ARG, "host buffer is NULL");
+    if (bytes != blin_state_bytes(st))
+        return fail(BLIN_ERR_STATE, "bytes=%zu but the state holds %zu", bytes, blin_state_bytes(st));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t sb = sizeof(float) * (size_t)st->B * st->H * st->d * st->d;
+    cudaError_t e = cudaMemcpyAsync(host, st->S, sb, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(static_cast<char *>(host) + sb, st->z, bytes - sb, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "state copy to host");
+    return BLIN_OK;
+}
+
+blin_status blin_state_copy_from_host(blin_state *st, const void *host, size_t bytes, int t_next,
+                                      blin_stream stream) {
+    blin_status rc = check_state(st);
+    if (rc != BLIN_OK) return rc;
+    if (host == nullptr) return fail(BLIN_ERR_INVALID_ARG, "host buffer is NULL");
+    if (t_next < 0) return fail(BLIN_ERR_INVALID_ARG, "t_next must be >= 0");
+    if (bytes != blin_state_bytes(st))
+        return fail(BLIN_ERR_STATE, "bytes=%zu but the state holds %zu", bytes, blin_state_bytes(st));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t sb = sizeof(float) * (size_t)st->B * st->H * st->d * st->d;
+    cudaError_t e = cudaMemcpyAsync(st->S, host, sb, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(st->z, static_cast<const char *>(host) + sb, bytes - sb, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "state copy from host");
+    st->t_next = t_next;
+    return BLIN_OK;
+}
+
+static blin_status ensure_scratch(blin_state *st, size_t need, cudaStream_t s) {
+    if (st->scratch_bytes >= need) return BLIN_OK;
+    void *p = nullptr;
+    cudaError_t e = cudaMallocAsync(&p, need, s);
+    if (e != cudaSuccess) return cuda_fail(e, "block-step scratch allocation");
+    if (st->scratch) cudaFreeAsync(st->scratch, s);
+    st->scratch = p;
+    st->scratch_bytes = need;
+    return BLIN_OK;
+}
+
+blin_status blin_state_reserve(blin_state *st, long max_block_tokens, blin_stream stream) {
+    blin_status rc = check_state(st);
+    if (rc != BLIN_OK) return rc;
+    if (max_block_tokens < 1 || max_block_tokens >= (1L << 30))
+        return fail(BLIN_ERR_INVALID_ARG, "max_block_tokens out of range");
+    // Widest table: all tokens on one axis of one frame (Hgt = 1, Wid = tokens).
+    const int split_wide[3] = {0, 0, st->d};
+    Plan p = make_plan(st->B, st->H, st->d, 1, 1, (int)max_block_tokens, 1, 0, true, split_wide, 0.f);
+    return ensure_scratch(st, plan_bytes(p), static_cast<cudaStream_t>(stream));
+}
+
+size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom *g) {
+    if (g == nullptr) return 0;
+    if (check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps) != BLIN_OK) return 0;
+    if (g->block_frames < 1) return 0;
+    Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, 0, false, g->rope_split, g->eps, true);
+    return plan_bytes(p);
+}
+
+blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
+                         int H, int d, const blin_geom *g, blin_state *st, void *workspace,
+                         size_t ws_bytes, blin_stream stream) {
+    if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
+    blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
+    if (rc != BLIN_OK) return rc;
+    if (g->block_frames < 1) return fail(BLIN_ERR_INVALID_ARG, "block_frames must be >= 1");
+    if ((rc = check_io(q, k, v, o, dt)) != BLIN_OK) return rc;
+    if (st != nullptr) {
+        if ((rc = check_state(st)) != BLIN_OK) return rc;
+        if (st->B != B || st->H != H || st->d != d)
+            return fail(BLIN_ERR_STATE, "state is B=%d H=%d d=%d, call is B=%d H=%d d=%d", st->B, st->H,
+                        st->d, B, H, d);
+    }
+    if (g->T == 0) return BLIN_OK;
+    const size_t need = blin_prefill_workspace_size(B, H, d, g);
+    if (workspace == nullptr || ws_bytes < need)
+        return fail(BLIN_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? ws_bytes : 0, need);
+    if (!aligned16(workspace)) return fail(BLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
+    const int t0 = st ? st->t_next : 0;
+    if ((long long)t0 + g->T >= (1LL << 30)) return fail(BLIN_ERR_SHAPE, "frame index overflow");
+    Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, t0, false, g->rope_split, g->eps);
+    plan_bind(p, workspace);
+    rc = run(p, q, k, v, o, dt, st ? st->S : nullptr, st ? st->z : nullptr, st ? st->S : nullptr,
+             st ? st->z : nullptr, (double)g->theta, g->rope_split, static_cast<cudaStream_t>(stream));
+    if (rc != BLIN_OK) return rc;
+    if (st) st->t_next += g->T;
+    return BLIN_OK;
+}
+
+blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
+                            int H, int d, int Hgt, int Wid, int frames, const int rope_split[3],
+                            float theta, float eps, blin_state *st, int commit, blin_stream stream) {
+    blin_status rc = check_common(B, H, d, frames, Hgt, Wid, rope_split, theta, eps);
+    if (rc != BLIN_OK) return rc;
+    if (frames < 1) return fail(BLIN_ERR_INVALID_ARG, "frames must be >= 1");
+    if (commit != 0 && commit != 1) return fail(BLIN_ERR_INVALID_ARG, "commit must be 0 or 1");
+    if ((rc = check_io(q, k, v, o, dt)) != BLIN_OK) return rc;
+    if ((rc = check_state(st)) != BLIN_OK) return rc;
+    if (st->B != B || st->H != H || st->d != d)
+        return fail(BLIN_ERR_STATE, "state is B=%d H=%d d=%d, call is B=%d H=%d d=%d", st->B, st->H, st->d,
+                    B, H, d);
+    if ((long long)st->t_next + frames >= (1LL << 30)) return fail(BLIN_ERR_SHAPE, "frame index overflow");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Plan p = make_plan(B, H, d, frames, Hgt, Wid, frames, st->t_next, true, rope_split, eps);
+    if ((rc = ensure_scratch(st, plan_bytes(p), s)) != BLIN_OK) return rc;
+    plan_bind(p, st->scratch);
+    rc = run(p, q, k, v, o, dt, st->S, st->z, commit ? st->S : nullptr, commit ? st->z : nullptr,
+             (double)theta, rope_split, s);
+    if (rc != BLIN_OK) return rc;
+    if (commit) st->t_next += frames;
+    return BLIN_OK;
+}
+
+blin_status blin_set_timing_events(void *const *events, int n) {
+    if (events != nullptr && n < 8) return fail(BLIN_ERR_INVALID_ARG, "need 8 events (got %d)", n);
+    g_timing = reinterpret_cast<cudaEvent_t const *>(events);
+    return BLIN_OK;
+}
+
+blin_status blin_device_status(int *code) {
+    int c = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "device synchronise");
+    e = read_and_clear_watchdog(&c);
+    if (e != cudaSuccess) return cuda_fail(e, "watchdog read");
+    if (code) *code = c;
+    if (c != 0) return fail(BLIN_ERR_DEVICE, "a kernel wait ran out (watchdog code %d)", c);
+    return BLIN_OK;
+}
+
+}  // extern "C"

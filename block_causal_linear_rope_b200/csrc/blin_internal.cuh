@@ -1,0 +1,72 @@
+// Internal declarations shared by the blin host layer and its kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace blin {
+
+// Tokens per TMA tile / MMA row block, tiles per state chunk and per output CTA.
+constexpr int kTile = 128;
+constexpr int kChunkTiles = 8;
+constexpr int kChunk = kTile * kChunkTiles;  // 1024 tokens: fixed per block => bit-exact streaming
+constexpr int kQTiles = 8;                    // output tiles per CTA
+
+// Geometry of one call, shared by all kernels of that call.
+struct KGeom {
+    int BH;               // B * H
+    int N;                // tokens per head in this call
+    int T, Hg, Wg, HW;    // latent grid of the call
+    int t0;               // absolute index of the call's first frame
+    int F;                // frames per full block
+    int first_end;        // relative frame at which block 0 ends
+    int nblk;             // blocks touched by the call
+    int cpb;              // state chunks per block (stride of the partial buffer)
+    int qcpb;             // output CTAs per block (grid.x of the output kernel)
+    int pt, py, px;       // RoPE pairs per axis (t, y, x)
+    float eps;
+    const float2 *tab;    // (cos, sin): [T][pt] then [Hg][py] then [Wg][px]
+    int tab_y, tab_x;     // offsets (in float2) of the y and x tables
+    float *part;          // [BH][nblk][cpb][d*d + d] chunk partial states
+    float *prefix;        // [BH][nblk][d*d + d] inclusive prefix states S_<=b, z_<=b
+};
+
+__host__ __device__ inline int block_frame_begin(const KGeom &g, int b) {
+    return b == 0 ? 0 : g.first_end + (b - 1) * g.F;
+}
+__host__ __device__ inline int block_frame_end(const KGeom &g, int b) {
+    int e = g.first_end + b * g.F;
+    return e < g.T ? e : g.T;
+}
+
+// Device-side watchdog word: 0 = fine, otherwise the code of the wait that ran out.
+enum WatchdogCode : int {
+    WD_NONE = 0,
+    WD_PARTIAL_FULL = 1,
+    WD_PARTIAL_EMPTY = 2,
+    WD_PARTIAL_ACC = 3,
+    WD_OUT_FULL = 11,
+    WD_OUT_EMPTY = 12,
+    WD_OUT_MMA = 13,
+};
+
+// Launchers (all enqueue on `s`; return the launch's cudaError_t).
+cudaError_t launch_rope_table(const KGeom &g, double theta, cudaStream_t s);
+cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
+                        float *z_out, cudaStream_t s);
+cudaError_t launch_partial_simt(const KGeom &g, int d, bool bf16, const void *k, const void *v,
+                                cudaStream_t s);
+cudaError_t launch_output_simt(const KGeom &g, int d, bool bf16, const void *q, void *o,
+                               cudaStream_t s);
+// Tensor-core path (bf16, d in {32, 64}, splits with a compiled variant).
+bool tc_supported(int d, const int split[3]);
+cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv,
+                              cudaStream_t s);
+cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo,
+                             void *o, cudaStream_t s);
+
+// Device watchdog access.
+cudaError_t read_and_clear_watchdog(int *code);
+
+}  // namespace blin

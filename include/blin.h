@@ -1,0 +1,189 @@
+/*
+ * blin — block-causal ReLU linear attention with 3D RoPE (numerator only) and
+ * a constant-size (S, z) cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (SANA-Video pages):
+ *   - "SANA-Video: Efficient Video Generation with Block Linear Diffusion
+ *     Transformer [ICLR 2026, Oral]" talk transcript, linear-attention state
+ *     review: the state is d x d whatever the sequence length; block i adds its
+ *     contribution K_i^T V_i to the cached state; block b attends to itself and
+ *     every earlier block; 3D RoPE is used inside linear attention.
+ *   - "四库全闻快报 ... SANA-Video" news article, positional-encoding paragraph:
+ *     RoPE is kept in the numerator and removed from the denominator.
+ *
+ * For one head, with phi = ReLU and R_n the 3D rotation at token n:
+ *   S_<=b = S_0 + sum_{m in blocks <= b} (R_m phi(k_m)) v_m^T      (d x d)
+ *   z_<=b = z_0 + sum_{m in blocks <= b} phi(k_m)                   (d)
+ *   o_n   = (R_n phi(q_n))^T S_<=b(n) / (phi(q_n) . z_<=b(n) + eps)
+ *
+ * Conventions (readings of points the pages leave open):
+ *   - Tensors are contiguous [B][H][N][d], d innermost; N = T * Hgt * Wid with
+ *     tokens ordered t-major, then y, then x.
+ *   - Frame t of a call has absolute index t_abs = t0 + t, t0 being the cache's
+ *     frame count (0 without a cache).  Blocks group F = block_frames absolute
+ *     frames: block(t_abs) = t_abs / F, so a call that starts inside a block
+ *     first finishes that block.  Attention is full inside a block.
+ *   - RoPE: rope_split = (d_t, d_y, d_x), even, summing to d.  Axis sections
+ *     are consecutive (t, then y, then x); pair (2j, 2j+1) of an axis section
+ *     turns by p_axis * theta^(-2j/d_axis) with p = (t_abs, y, x).
+ *   - No 1/sqrt(d) scale.  eps is added after the denominator's dot product.
+ *   - States are fp32: S[B][H][d][d] (row = rotated key feature, column =
+ *     value feature) and z[B][H][d].  Outputs have the input dtype.
+ *
+ * Ownership: the caller owns q, k, v, o and any workspace (device memory).
+ * The library owns a state's S, z and block-step scratch, allocated in
+ * blin_state_init / blin_state_reserve / the first blin_block_step that needs
+ * more scratch, and freed in blin_state_free.  All work is enqueued
+ * asynchronously on the given stream (a cudaStream_t; NULL = legacy default).
+ *
+ * Errors: arguments are checked on the host before any launch; a check that
+ * fails returns a negative blin_status and sets a thread-local message
+ * (blin_last_error).  CUDA launch failures return BLIN_ERR_CUDA.  Kernel
+ * waits are bounded: a wait that exceeds its limit records a code readable by
+ * blin_device_status and the kernel returns instead of hanging.
+ */
+#ifndef BLIN_H
+#define BLIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BLIN_API __attribute__((visibility("default")))
+#else
+#define BLIN_API
+#endif
+
+typedef void *blin_stream; /* a cudaStream_t */
+
+typedef enum {
+    BLIN_OK = 0,
+    BLIN_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, bad flag, eps/theta out of range */
+    BLIN_ERR_SHAPE = -2,       /* d not 32/64, bad rope split, frames > block_frames, size overflow */
+    BLIN_ERR_DTYPE = -3,       /* unknown dtype */
+    BLIN_ERR_ALIGN = -4,       /* q/k/v/o/workspace not 16-byte aligned */
+    BLIN_ERR_WORKSPACE = -5,   /* workspace too small */
+    BLIN_ERR_STATE = -6,       /* freed/foreign state, B/H/d mismatch, wrong device, wrong byte count */
+    BLIN_ERR_CUDA = -7,        /* a CUDA runtime/driver call failed */
+    BLIN_ERR_DEVICE = -8       /* a kernel's bounded wait ran out (see blin_device_status) */
+} blin_status;
+
+typedef enum { BLIN_F32 = 0, BLIN_BF16 = 1 } blin_dtype;
+
+/* Latent grid and method constants of one call.
+ *   T, Hgt, Wid   latent frames, height and width of this call (N = T*Hgt*Wid)
+ *   block_frames  F, latent frames per causal block (>= 1)
+ *   rope_split    dims of the t, y, x RoPE sections (even, sum = d)
+ *   theta         RoPE base (> 0), eps  denominator offset (>= 0, finite) */
+typedef struct {
+    int T, Hgt, Wid;
+    int block_frames;
+    int rope_split[3];
+    float theta;
+    float eps;
+} blin_geom;
+
+typedef struct blin_state blin_state; /* opaque (S, z) cache on one device */
+
+/* ---------------------------------------------------------------- state */
+
+/* Allocate a zeroed cache S[B][H][d][d], z[B][H][d] (fp32) on the current
+ * device, t_next = 0.  Memory stays constant however many blocks pass through
+ * it (talk transcript: constant KV-cache memory for any video length). */
+BLIN_API blin_status blin_state_init(int B, int H, int d, blin_stream stream, blin_state **out);
+
+/* Free the cache and its scratch (synchronises the device).  NULL is a no-op. */
+BLIN_API blin_status blin_state_free(blin_state *st);
+
+/* Zero S and z (on stream) and set t_next = 0. */
+BLIN_API blin_status blin_state_reset(blin_state *st, blin_stream stream);
+
+/* Device pointers of S and z and the next absolute frame index.  Any output
+ * pointer may be NULL.  The pointers stay valid until blin_state_free. */
+BLIN_API blin_status blin_state_tensors(const blin_state *st, float **S, float **z, int *t_next);
+
+/* Bytes of one host copy of the cache: B*H*(d*d + d)*4 (S then z). */
+BLIN_API size_t blin_state_bytes(const blin_state *st);
+
+/* Copy S then z into host memory (bytes must equal blin_state_bytes).  The
+ * copy is enqueued on stream; synchronise before reading host. */
+BLIN_API blin_status blin_state_copy_to_host(const blin_state *st, void *host, size_t bytes, blin_stream stream);
+
+/* Restore S then z from host memory and set t_next (checkpoint resume).  The
+ * host buffer must stay valid until the stream reaches the copy. */
+BLIN_API blin_status blin_state_copy_from_host(blin_state *st, const void *host, size_t bytes, int t_next,
+                                      blin_stream stream);
+
+/* Pre-size the block-step scratch for blocks of up to max_block_tokens tokens
+ * (Hgt*Wid*frames), so that later blin_block_step calls allocate nothing
+ * (for instance before capturing them in a CUDA graph). */
+BLIN_API blin_status blin_state_reserve(blin_state *st, long max_block_tokens, blin_stream stream);
+
+/* ---------------------------------------------------------------- prefill */
+
+/* Workspace bytes blin_prefill needs for this shape (0 on invalid input). */
+BLIN_API size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom *g);
+
+/* Block-causal linear attention over a whole latent video (or a continuation).
+ *   q, k, v  device [B][H][N][d] of dtype dt;  o  device [B][H][N][d] output
+ *   st       optional cache.  NULL: start from S = 0, z = 0, t0 = 0.
+ *            Otherwise start from its (S, z) with t0 = its t_next, and on
+ *            return (in stream order) it holds the final (S, z) with
+ *            t_next += T.
+ *   workspace device scratch of at least blin_prefill_workspace_size bytes,
+ *            16-byte aligned; contents on entry are ignored.
+ * T = 0 is valid and does nothing.  The result for every row is independent of
+ * how the same frames are split into calls, and the final (S, z) is bitwise
+ * equal to the one blin_block_step reaches over the same blocks. */
+BLIN_API blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
+                         int B, int H, int d, const blin_geom *g, blin_state *st,
+                         void *workspace, size_t ws_bytes, blin_stream stream);
+
+/* ---------------------------------------------------------------- decode */
+
+/* One autoregressive block (talk transcript, block-causal walk-through: the
+ * new block reads the cached state plus its own contribution; the sum is
+ * cached for the next block).
+ *   q, k, v, o  device [B][H][frames*Hgt*Wid][d] of dtype dt
+ *   frames      latent frames in this block, 1..block_frames of the caller's
+ *               schedule (the library treats the whole call as one block)
+ *   commit      1: S += block K~^T V, z += sum phi(k), t_next += frames.
+ *               0: read-only pass (a denoising step of the same block);
+ *                  the cache is left unchanged.
+ * Positions continue from the cache: t_abs = t_next + t.  Needs scratch owned
+ * by the state; the first call with a larger block grows it (allocation on
+ * stream), blin_state_reserve avoids that. */
+BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
+                            int B, int H, int d, int Hgt, int Wid, int frames,
+                            const int rope_split[3], float theta, float eps,
+                            blin_state *st, int commit, blin_stream stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Thread-local message for the last non-OK status of this thread ("" if none). */
+BLIN_API const char *blin_last_error(void);
+
+/* Read (synchronously) and clear the current device's kernel watchdog word:
+ * 0 = no bounded wait ran out since the last call; otherwise a code naming the
+ * wait that gave up.  Returns BLIN_ERR_DEVICE when the word was non-zero. */
+BLIN_API blin_status blin_device_status(int *code);
+
+/* Per-launch timing (profiling aid).  When `events` is non-NULL, the calling
+ * thread's next blin_prefill / blin_block_step calls record events[2*i] just
+ * before and events[2*i+1] just after launch i on the call's stream, for
+ * i = 0 RoPE table, 1 partial states, 2 block scan, 3 output (n >= 8
+ * cudaEvent_t handles, owned by the caller).  NULL turns recording off. */
+BLIN_API blin_status blin_set_timing_events(void *const *events, int n);
+
+/* Library version string. */
+BLIN_API const char *blin_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLIN_H */

@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: symbols, sizes and host-side argument validation.
+
+Every call here returns before any CUDA launch (the checks run first), so the
+library can be exercised on a machine without a device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_causal_linear_rope_b200 as blin
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "blin.h")
+
+OK, INVALID, SHAPE, DTYPE, ALIGN, WORKSPACE, STATE = 0, -1, -2, -3, -4, -5, -6
+FAKE = 1 << 20  # a 16-byte aligned non-NULL address that is never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(blin_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["blin_state_init", "blin_state_free", "blin_prefill", "blin_block_step",
+                 "blin_prefill_workspace_size", "blin_last_error", "blin_state_copy_to_host",
+                 "blin_state_copy_from_host", "blin_state_tensors", "blin_state_reset"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    for name in declared_functions():
+        assert hasattr(blin.lib, name), name
+
+
+def test_library_exports_nothing_else():
+    out = subprocess.run(["nm", "-D", "--defined-only", blin.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    ours = {s for s in exported if s.startswith("blin_")}
+    assert ours == set(declared_functions())
+
+
+def geom(T=21, Hg=30, Wg=52, F=3, split=(8, 12, 12), theta=1e4, eps=1e-6):
+    return blin._geom(T, Hg, Wg, F, split, theta, eps)
+
+
+def ws(B, H, d, g):
+    return blin.lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g))
+
+
+def test_workspace_size_formula():
+    # tables + partials + prefix states, each padded to 256 B, plus 256 B of alignment slack
+    B, H, d = 1, 70, 32
+    g = geom()
+    E = d * d + d
+    nblk = 21 // 3 + 1
+    cpb = -(-(3 * 30 * 52) // 1024)
+    pad = lambda x: (x + 255) // 256 * 256
+    want = 256 + pad(8 * (21 * 4 + 30 * 6 + 52 * 6 + 1)) + pad(4 * B * H * nblk * cpb * E) + pad(4 * B * H * nblk * E)
+    assert ws(B, H, d, g) == want
+
+
+def test_workspace_size_rejects_bad_shapes():
+    assert ws(1, 70, 48, geom()) == 0
+    assert ws(1, 70, 32, geom(split=(8, 12, 10))) == 0
+    assert ws(1, 70, 32, geom(split=(7, 13, 12))) == 0
+    assert ws(0, 70, 32, geom()) == 0
+    assert ws(1, 70, 32, geom(F=0)) == 0
+    assert ws(1, 70, 32, geom(theta=0.0)) == 0
+    assert ws(1, 70, 32, geom(eps=-1.0)) == 0
+
+
+def prefill_raw(q=FAKE, k=FAKE, v=FAKE, o=FAKE, dt=1, B=1, H=2, d=32, g=None, st=None, w=FAKE, wb=1 << 30):
+    g = g or geom(T=4, Hg=4, Wg=4)
+    return blin.lib.blin_prefill(q, k, v, o, dt, B, H, d, ctypes.byref(g), st, w, wb, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(o=None), INVALID), (dict(dt=7), DTYPE), (dict(d=48), SHAPE),
+    (dict(q=FAKE + 8), ALIGN), (dict(w=None), WORKSPACE), (dict(wb=16), WORKSPACE),
+    (dict(w=FAKE + 4), ALIGN), (dict(B=0), INVALID),
+    (dict(g=geom(T=4, Hg=4, Wg=4, split=(8, 8, 8))), SHAPE),
+    (dict(g=geom(T=4, Hg=0, Wg=4)), INVALID), (dict(g=geom(T=4, Hg=4, Wg=4, F=0)), INVALID),
+    (dict(g=geom(T=4, Hg=4, Wg=4, eps=float("nan"))), INVALID),
+])
+def test_prefill_rejects_bad_arguments_before_launch(kw, code):
+    assert prefill_raw(**kw) == code
+    assert blin.lib.blin_last_error().decode() != ""
+
+
+def test_prefill_with_no_frames_is_a_no_op():
+    assert prefill_raw(g=geom(T=0, Hg=4, Wg=4), w=None, wb=0) == OK
+
+
+def test_geom_null_and_state_null():
+    assert blin.lib.blin_prefill(FAKE, FAKE, FAKE, FAKE, 1, 1, 2, 32, None, None, FAKE, 1 << 20, None) == INVALID
+    split = (ctypes.c_int * 3)(8, 12, 12)
+    rc = blin.lib.blin_block_step(FAKE, FAKE, FAKE, FAKE, 1, 1, 2, 32, 4, 4, 3, ctypes.byref(split), 1e4, 1e-6,
+                                  None, 1, None)
+    assert rc == INVALID
+
+
+def test_block_step_argument_checks():
+    split = (ctypes.c_int * 3)(8, 12, 12)
+    bad = (ctypes.c_int * 3)(8, 12, 14)
+    call = lambda **kw: blin.lib.blin_block_step(
+        kw.get("q", FAKE), FAKE, FAKE, FAKE, kw.get("dt", 1), 1, 2, kw.get("d", 32), 4, 4, kw.get("frames", 3),
+        ctypes.byref(kw.get("split", split)), 1e4, 1e-6, FAKE, kw.get("commit", 1), None)
+    assert call(frames=0) == INVALID
+    assert call(split=bad) == SHAPE
+    assert call(commit=2) == INVALID
+    assert call(dt=5) == DTYPE
+    assert call(q=FAKE + 2) == ALIGN
+
+
+def test_state_accessors_reject_null():
+    assert blin.lib.blin_state_tensors(None, None, None, None) == INVALID
+    assert blin.lib.blin_state_bytes(None) == 0
+    assert blin.lib.blin_state_free(None) == OK
+    out = ctypes.c_void_p()
+    assert blin.lib.blin_state_init(1, 1, 40, None, ctypes.byref(out)) == SHAPE
+    assert blin.lib.blin_state_init(0, 1, 32, None, ctypes.byref(out)) == INVALID
+    assert blin.lib.blin_state_init(1, 1, 32, None, None) == INVALID
+
+
+def test_version_string():
+    assert b"sm_100a" in blin.lib.blin_version()
