@@ -102,15 +102,16 @@ bool tc_supported(int d, const int split[3]) {
     return false;
 }
 
-// Raise the dynamic shared-memory limit of a kernel once per device.
-template <typename KernelT>
-static cudaError_t set_smem(KernelT kernel, int bytes) {
+// Raise the dynamic shared-memory limit of a kernel once per device (one cache
+// per kernel: the template parameter is the kernel itself, not its type).
+template <auto Kernel>
+static cudaError_t set_smem(int bytes) {
     static bool done[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
     return e;
 }
@@ -124,12 +125,12 @@ cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, cons
     if (d == 32) {
         auto k = partial_tc_kernel<32, 4, 6, 6>;
         constexpr int smem = partial_tc_smem_bytes<32>();
-        if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+        if ((e = set_smem<partial_tc_kernel<32, 4, 6, 6>>(smem)) != cudaSuccess) return e;
         k<<<grid, 160, smem, s>>>(mk, mv, g, wd);
     } else {
         auto k = partial_tc_kernel<64, 8, 12, 12>;
         constexpr int smem = partial_tc_smem_bytes<64>();
-        if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+        if ((e = set_smem<partial_tc_kernel<64, 8, 12, 12>>(smem)) != cudaSuccess) return e;
         k<<<grid, 160, smem, s>>>(mk, mv, g, wd);
     }
     return cudaGetLastError();
@@ -145,12 +146,12 @@ cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const
     if (d == 32) {
         auto k = output_tc_kernel<32, 4, 6, 6>;
         constexpr int smem = output_tc_smem_bytes<32>();
-        if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+        if ((e = set_smem<output_tc_kernel<32, 4, 6, 6>>(smem)) != cudaSuccess) return e;
         k<<<grid, 160, smem, s>>>(mq, mo, g, ob, wd);
     } else {
         auto k = output_tc_kernel<64, 8, 12, 12>;
         constexpr int smem = output_tc_smem_bytes<64>();
-        if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+        if ((e = set_smem<output_tc_kernel<64, 8, 12, 12>>(smem)) != cudaSuccess) return e;
         k<<<grid, 160, smem, s>>>(mq, mo, g, ob, wd);
     }
     return cudaGetLastError();

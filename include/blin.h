@@ -136,9 +136,11 @@ BLIN_API size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom
  *            t_next += T.
  *   workspace device scratch of at least blin_prefill_workspace_size bytes,
  *            16-byte aligned; contents on entry are ignored.
- * T = 0 is valid and does nothing.  The result for every row is independent of
- * how the same frames are split into calls, and the final (S, z) is bitwise
- * equal to the one blin_block_step reaches over the same blocks. */
+ * T = 0 is valid and does nothing.  Splitting the frames into several calls
+ * at block boundaries gives the same rows as one call, and the final (S, z) is
+ * bitwise equal to the one blin_block_step reaches over the same blocks.  A
+ * call that ends inside a block lets that block's rows see only the frames
+ * given so far; the next call's rows of the same block see the whole block. */
 BLIN_API blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                          int B, int H, int d, const blin_geom *g, blin_state *st,
                          void *workspace, size_t ws_bytes, blin_stream stream);
