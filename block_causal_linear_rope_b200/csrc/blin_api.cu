@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/blin.h"
@@ -111,6 +112,16 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
     g.eps = eps;
     g.tab_y = T * g.pt;
     g.tab_x = g.tab_y + Hg * g.py;
+    // chunks of one head: sum over blocks of ceil(block tokens / chunk)
+    long long chunks = 0;
+    for (int b = 0; b < g.nblk && !for_size; ++b)
+        chunks += ((long long)(block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
+    g.chunks_per_bh = (int)chunks;
+    // The persistent kernels keep the call's whole RoPE table in shared memory
+    // when it is small; otherwise they read it from global memory.
+    const long long tab_entries = (long long)T * g.pt + (long long)Hg * g.py + (long long)Wg * g.px;
+    g.tab_smem_bytes = (int)std::min<long long>(tab_entries * (long long)sizeof(float2), 1 << 30);
+    g.tab_smem = g.tab_smem_bytes <= tc_table_smem_limit() ? 1 : 0;
     const size_t E = (size_t)d * d + d;
     p.tab_bytes = align256(sizeof(float2) * ((size_t)T * g.pt + (size_t)Hg * g.py + (size_t)Wg * g.px + 1));
     p.part_bytes = align256(sizeof(float) * (size_t)g.BH * g.nblk * g.cpb * E);
@@ -171,9 +182,14 @@ static void mark(int i, bool after, cudaStream_t s) {
 static blin_status run(Plan &p, const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                        const float *S_in, const float *z_in, float *S_out, float *z_out, double theta,
                        const int split[3], cudaStream_t s) {
+    p.g.S_in = S_in;
+    p.g.z_in = z_in;
+    p.g.theta = theta;
+    p.g.S_out = S_out;
+    p.g.z_out = z_out;
     const KGeom &g = p.g;
     const int d = p.d;
-    const bool tc = dt == BLIN_BF16 && tc_supported(d, split);
+    const bool tc = dt == BLIN_BF16 && tc_supported(d, split) && g.tab_smem;
     CUtensorMap mq, mk, mv, mo;
     if (tc) {
         const long long rows = (long long)g.BH * g.N;
@@ -184,7 +200,8 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
     const bool bf = dt == BLIN_BF16;
     cudaError_t e;
     mark(0, false, s);
-    if ((e = launch_rope_table(g, theta, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
+    // the tensor-core kernels build their RoPE tables in shared memory themselves
+    if (!tc && (e = launch_rope_table(g, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
     mark(0, true, s);
     mark(1, false, s);
     e = tc ? launch_partial_tc(g, d, mk, mv, s) : launch_partial_simt(g, d, bf, k, v, s);

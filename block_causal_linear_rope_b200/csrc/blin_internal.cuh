@@ -30,6 +30,12 @@ struct KGeom {
     int tab_y, tab_x;     // offsets (in float2) of the y and x tables
     float *part;          // [BH][nblk][cpb][d*d + d] chunk partial states
     float *prefix;        // [BH][nblk][d*d + d] inclusive prefix states S_<=b, z_<=b
+    int chunks_per_bh;    // state chunks of one head in this call
+    double theta;         // RoPE base
+    int tab_smem;         // 1: the RoPE table fits the tensor-core kernels' shared memory
+    int tab_smem_bytes;   // bytes of the whole table (t, y and x parts)
+    const float *S_in, *z_in;  // cache entering the call (NULL: zero)
+    float *S_out, *z_out;      // cache after the call (NULL: not written)
 };
 
 __host__ __device__ inline int block_frame_begin(const KGeom &g, int b) {
@@ -46,13 +52,18 @@ enum WatchdogCode : int {
     WD_PARTIAL_FULL = 1,
     WD_PARTIAL_EMPTY = 2,
     WD_PARTIAL_ACC = 3,
+    WD_PARTIAL_READY = 4,
     WD_OUT_FULL = 11,
     WD_OUT_EMPTY = 12,
     WD_OUT_MMA = 13,
+    WD_OUT_READY = 14,
+    WD_OUT_ACCE = 15,
+    WD_OUT_BREADY = 16,
 };
 
 // Launchers (all enqueue on `s`; return the launch's cudaError_t).
-cudaError_t launch_rope_table(const KGeom &g, double theta, cudaStream_t s);
+// Fills the RoPE table in global memory (CUDA-core path).
+cudaError_t launch_rope_table(const KGeom &g, cudaStream_t s);
 cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
                         float *z_out, cudaStream_t s);
 cudaError_t launch_partial_simt(const KGeom &g, int d, bool bf16, const void *k, const void *v,
@@ -61,8 +72,12 @@ cudaError_t launch_output_simt(const KGeom &g, int d, bool bf16, const void *q, 
                                cudaStream_t s);
 // Tensor-core path (bf16, d in {32, 64}, splits with a compiled variant).
 bool tc_supported(int d, const int split[3]);
+// Partial states plus the fused per-head scan (writes prefix and S_out/z_out).
 cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv,
                               cudaStream_t s);
+// Shared-memory bytes the tensor-core kernels need for a RoPE table copy of
+// `entries` float2 (0 when the table is read from global memory).
+int tc_table_smem_limit();
 cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo,
                              void *o, cudaStream_t s);
 

@@ -2,6 +2,8 @@
 // per device, no relocatable device code needed) together with its launchers.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "blin_internal.cuh"
 
 namespace blin {
@@ -33,21 +35,13 @@ static int *watchdog_ptr() {
     return ptrs[dev];
 }
 
-cudaError_t launch_rope_table(const KGeom &g, double theta, cudaStream_t s) {
+cudaError_t launch_rope_table(const KGeom &g, cudaStream_t s) {
     const int total = g.T * g.pt + g.Hg * g.py + g.Wg * g.px;
     if (total == 0) return cudaSuccess;
     const int threads = 256;
     const int blocks = (total + threads - 1) / threads;
-    rope_table_kernel<<<blocks, threads, 0, s>>>(const_cast<float2 *>(g.tab), g.T, g.t0, g.Hg, g.Wg,
-                                                 g.pt, g.py, g.px, theta);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
-                        float *z_out, cudaStream_t s) {
-    const int E = d * d + d;
-    dim3 grid((E + 255) / 256, g.BH);
-    scan_kernel<<<grid, 256, 0, s>>>(g, d, S_in, z_in, S_out, z_out);
+    rope_table_kernel<<<blocks, threads, 0, s>>>(const_cast<float2 *>(g.tab), g.T, g.t0, g.Hg, g.Wg, g.pt, g.py,
+                                                 g.px, g.theta);
     return cudaGetLastError();
 }
 
@@ -102,59 +96,106 @@ bool tc_supported(int d, const int split[3]) {
     return false;
 }
 
-// Raise the dynamic shared-memory limit of a kernel once per device (one cache
-// per kernel: the template parameter is the kernel itself, not its type).
+// Raise the dynamic shared-memory limit of a kernel (cached per device and
+// kernel: the template parameter is the kernel itself, not its type).
 template <auto Kernel>
 static cudaError_t set_smem(int bytes) {
-    static bool done[64] = {false};
+    static int done[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+    if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 227 * 1024;
     return e;
+}
+
+int tc_table_smem_limit() { return 24 * 1024; }
+
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel in the stream finishes; it calls
+// griddepcontrol.wait before reading anything that kernel wrote.
+// `pdl` false gives an ordinary launch (the first kernel of a call, which reads
+// the caller's inputs, always waits for everything before it).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_ex(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
+                             Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
+                              Args &&...args) {
+    return launch_ex(true, kernel, grid, block, smem, s, std::forward<Args>(args)...);
+}
+
+cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
+                        float *z_out, cudaStream_t s) {
+    const int E4 = (d * d + d) / 4;
+    const dim3 grid((E4 + kScanSlice - 1) / kScanSlice, g.BH);
+    const int groups = g.nblk < 32 ? (g.nblk > 0 ? g.nblk : 1) : 32;  // thread groups of 32 columns
+    cudaError_t e = launch_pdl(scan_kernel, grid, dim3(kScanSlice * groups), 0, s, g, d, S_in, z_in, S_out, z_out);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Persistent grid: as many CTAs as fit on the device at once, never more than
+// there are work units.
+template <auto Kernel>
+static int persistent_grid(int smem, int threads, long long units) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 1;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, Kernel, threads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const long long n = (long long)sms * per_sm;
+    return (int)(units < n ? (units > 0 ? units : 1) : n);
+}
+
+template <auto Kernel, typename... Args>
+static cudaError_t launch_persistent(bool pdl, int smem, int threads, long long units, cudaStream_t s,
+                                     Args &&...args) {
+    cudaError_t e = set_smem<Kernel>(smem);
+    if (e != cudaSuccess) return e;
+    const int grid = persistent_grid<Kernel>(smem, threads, units);
+    e = launch_ex(pdl, Kernel, dim3(grid), dim3(threads), smem, s, std::forward<Args>(args)...);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv,
                               cudaStream_t s) {
     int *wd = watchdog_ptr();
     if (wd == nullptr) return cudaErrorInvalidDevice;
-    dim3 grid(g.cpb, g.nblk, g.BH);
-    cudaError_t e;
-    if (d == 32) {
-        auto k = partial_tc_kernel<32, 4, 6, 6>;
-        constexpr int smem = partial_tc_smem_bytes<32>();
-        if ((e = set_smem<partial_tc_kernel<32, 4, 6, 6>>(smem)) != cudaSuccess) return e;
-        k<<<grid, 160, smem, s>>>(mk, mv, g, wd);
-    } else {
-        auto k = partial_tc_kernel<64, 8, 12, 12>;
-        constexpr int smem = partial_tc_smem_bytes<64>();
-        if ((e = set_smem<partial_tc_kernel<64, 8, 12, 12>>(smem)) != cudaSuccess) return e;
-        k<<<grid, 160, smem, s>>>(mk, mv, g, wd);
-    }
-    return cudaGetLastError();
+    const long long units = (long long)g.cpb * g.nblk * g.BH;
+    const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
+    if (d == 32)
+        return launch_persistent<partial_tc_kernel<32, 4, 6, 6>>(false, P1<32>::FIXED + tab, P1<32>::THREADS, units, s, mk, mv, g, wd);
+    return launch_persistent<partial_tc_kernel<64, 8, 12, 12>>(false, P1<64>::FIXED + tab, P1<64>::THREADS, units, s, mk, mv, g, wd);
 }
 
 cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo,
                              void *o, cudaStream_t s) {
     int *wd = watchdog_ptr();
     if (wd == nullptr) return cudaErrorInvalidDevice;
-    dim3 grid(g.qcpb, g.nblk, g.BH);
-    cudaError_t e;
+    const long long units = (long long)g.qcpb * g.nblk * g.BH;
+    const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
     __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
-    if (d == 32) {
-        auto k = output_tc_kernel<32, 4, 6, 6>;
-        constexpr int smem = output_tc_smem_bytes<32>();
-        if ((e = set_smem<output_tc_kernel<32, 4, 6, 6>>(smem)) != cudaSuccess) return e;
-        k<<<grid, 160, smem, s>>>(mq, mo, g, ob, wd);
-    } else {
-        auto k = output_tc_kernel<64, 8, 12, 12>;
-        constexpr int smem = output_tc_smem_bytes<64>();
-        if ((e = set_smem<output_tc_kernel<64, 8, 12, 12>>(smem)) != cudaSuccess) return e;
-        k<<<grid, 160, smem, s>>>(mq, mo, g, ob, wd);
-    }
-    return cudaGetLastError();
+    if (d == 32)
+        return launch_persistent<output_tc_kernel<32, 4, 6, 6>>(true, P2<32>::FIXED + tab, P2<32>::THREADS, units, s, mq, mo, g, ob, wd);
+    return launch_persistent<output_tc_kernel<64, 8, 12, 12>>(true, P2<64>::FIXED + tab, P2<64>::THREADS, units, s, mq, mo, g, ob, wd);
 }
 
 }  // namespace blin

@@ -9,36 +9,40 @@
 namespace blin {
 
 // ---------------------------------------------------------------- RoPE table
-// (cos, sin) of p_axis * theta^(-2j/d_axis) for every position of the call:
-// [T][pt] (absolute frames t0..t0+T-1), then [Hg][py], then [Wg][px].
-// Angles and sin/cos are taken in double, then rounded to float.
-// (3D RoPE for linear attention: SANA-Video talk transcript.)
+// Entry i of the (cos, sin) table of a call: [T][pt] (absolute frames
+// t0..t0+T-1), then [Hg][py], then [Wg][px]; pair j of an axis with d_a dims
+// turns by p * theta^(-2j/d_a).  Angle and sin/cos are taken in double, then
+// rounded to float.  (3D RoPE for linear attention: SANA-Video talk transcript.)
+__device__ __forceinline__ float2 rope_entry(int i, int T, int t0, int Hg, int pt, int py, int px, double theta) {
+    const int nt = T * pt, ny = Hg * py;
+    int pos, j, pairs;
+    if (i < nt) {
+        pos = t0 + i / pt;
+        j = i % pt;
+        pairs = pt;
+    } else if (i < nt + ny) {
+        const int r = i - nt;
+        pos = r / py;
+        j = r % py;
+        pairs = py;
+    } else {
+        const int r = i - nt - ny;
+        pos = r / px;
+        j = r % px;
+        pairs = px;
+    }
+    const double freq = pow(theta, -2.0 * static_cast<double>(j) / static_cast<double>(2 * pairs));
+    double s, c;
+    sincos(static_cast<double>(pos) * freq, &s, &c);
+    return make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+// Whole table in global memory (CUDA-core path).
 __global__ void rope_table_kernel(float2 *tab, int T, int t0, int Hg, int Wg, int pt, int py, int px,
                                   double theta) {
-    const int nt = T * pt, ny = Hg * py, nx = Wg * px;
-    const int total = nt + ny + nx;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-        int pos, j, pairs;
-        if (i < nt) {
-            pos = t0 + i / pt;
-            j = i % pt;
-            pairs = pt;
-        } else if (i < nt + ny) {
-            const int r = i - nt;
-            pos = r / py;
-            j = r % py;
-            pairs = py;
-        } else {
-            const int r = i - nt - ny;
-            pos = r / px;
-            j = r % px;
-            pairs = px;
-        }
-        const double freq = pow(theta, -2.0 * static_cast<double>(j) / static_cast<double>(2 * pairs));
-        double s, c;
-        sincos(static_cast<double>(pos) * freq, &s, &c);
-        tab[i] = make_float2(static_cast<float>(c), static_cast<float>(s));
-    }
+    const int total = T * pt + Hg * py + Wg * px;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x)
+        tab[i] = rope_entry(i, T, t0, Hg, pt, py, px, theta);
 }
 
 // ---------------------------------------------------------------- block scan
@@ -49,28 +53,65 @@ __global__ void rope_table_kernel(float2 *tab, int T, int t0, int Hg, int Wg, in
 // The order depends only on the block's own length, so a block-by-block
 // stream reproduces a one-shot prefill bit for bit.  (Talk transcript: the
 // new state is the cached state plus the block's contribution.)
-__global__ void scan_kernel(KGeom g, int d, const float *S_in, const float *z_in, float *S_out,
-                            float *z_out) {
-    const int E = d * d + d;
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
-    const int bh = blockIdx.y;
-    if (e >= E) return;
-    float acc = 0.0f;
-    if (S_in != nullptr) acc = e < d * d ? S_in[(size_t)bh * d * d + e] : z_in[(size_t)bh * d + e - d * d];
-    for (int b = 0; b < g.nblk; ++b) {
-        const int ntok = (block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW;
-        const int nch = (ntok + kChunk - 1) / kChunk;
-        const float *p = g.part + ((size_t)(bh * g.nblk + b) * g.cpb) * E + e;
-        float pb = p[0];
-        for (int c = 1; c < nch; ++c) pb += p[(size_t)c * E];
-        acc = acc + pb;
-        g.prefix[((size_t)bh * g.nblk + b) * E + e] = acc;
+// One CTA per (head, 32 float4 columns): thread groups form the block sums
+// P_b in parallel (their chunk loads all in flight), then one group runs the
+// chain over blocks from shared memory.  Blocks are taken kScanSeg at a time.
+constexpr int kScanSlice = 32;  // float4 columns per CTA
+constexpr int kScanBatch = 8;   // chunk loads issued together per block
+constexpr int kScanSeg = 64;    // blocks staged in shared memory at once (32 KB)
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(KGeom g, int d, const float *S_in, const float *z_in,
+                                                    float *S_out, float *z_out) {
+    __shared__ float4 sm[kScanSeg * kScanSlice];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // chunk partials come from the previous kernel
+    const int E4 = (d * d + d) / 4;
+    const int bh = blockIdx.y, col = threadIdx.x % kScanSlice, grp = threadIdx.x / kScanSlice;
+    const int ngrp = blockDim.x / kScanSlice;
+    const int e4 = blockIdx.x * kScanSlice + col;
+    const bool live = e4 < E4;
+    const float4 *part = reinterpret_cast<const float4 *>(g.part);
+    float4 *prefix = reinterpret_cast<float4 *>(g.prefix);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (grp == 0 && live && S_in != nullptr)
+        acc = 4 * e4 < d * d ? reinterpret_cast<const float4 *>(S_in + (size_t)bh * d * d)[e4]
+                             : reinterpret_cast<const float4 *>(z_in + (size_t)bh * d)[e4 - d * d / 4];
+    for (int b0 = 0; b0 < g.nblk; b0 += kScanSeg) {
+        const int nb = min(kScanSeg, g.nblk - b0);
+        for (int bl = grp; bl < nb; bl += ngrp) {
+            if (!live) continue;
+            const int b = b0 + bl;
+            const int n = ((block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
+            const float4 *p = part + ((size_t)(bh * g.nblk + b) * g.cpb) * E4 + e4;
+            float4 v[kScanBatch];
+#pragma unroll
+            for (int c = 0; c < kScanBatch; ++c)
+                if (c < n) v[c] = __ldcg(p + (size_t)c * E4);
+            float4 pb = v[0];
+#pragma unroll
+            for (int c = 1; c < kScanBatch; ++c)
+                if (c < n) pb = f4add(pb, v[c]);
+            for (int c = kScanBatch; c < n; ++c) pb = f4add(pb, __ldcg(p + (size_t)c * E4));
+            sm[bl * kScanSlice + col] = pb;
+        }
+        __syncthreads();
+        if (grp == 0 && live) {
+            for (int bl = 0; bl < nb; ++bl) {
+                acc = f4add(acc, sm[bl * kScanSlice + col]);
+                prefix[((size_t)bh * g.nblk + b0 + bl) * E4 + e4] = acc;
+            }
+        }
+        __syncthreads();
     }
-    if (S_out != nullptr) {
-        if (e < d * d)
-            S_out[(size_t)bh * d * d + e] = acc;
+    if (grp == 0 && live && S_out != nullptr) {
+        if (4 * e4 < d * d)
+            reinterpret_cast<float4 *>(S_out + (size_t)bh * d * d)[e4] = acc;
         else
-            z_out[(size_t)bh * d + e - d * d] = acc;
+            reinterpret_cast<float4 *>(z_out + (size_t)bh * d)[e4 - d * d / 4] = acc;
     }
 }
 

@@ -1,22 +1,31 @@
 // Tensor-core path for bf16 Q/K/V on sm_100a (d = 32 or 64).
 //
-// Pass 1 (partial_tc_kernel): per (chunk of <= 1024 tokens, block, head) a CTA
-//   streams 128-token K and V tiles into shared memory with TMA (64B/128B
-//   swizzle), overwrites each K row in place with R_m phi(k_m) (bf16),
-//   accumulates phi(k_m) in fp32 registers, and lets tcgen05.mma accumulate
-//   P = K~^T V in TMEM (M = 64 rows of K~^T, N = d columns of V, K = tokens).
-//   Both operands are MN-major views of the token-major tiles, so no
-//   transpose is ever materialised.
-// Pass 2 (output_tc_kernel): per (up to 8 tiles of 128 queries, block, head)
-//   the CTA converts S_<=b to a bf16 K-major B operand once, streams Q tiles
-//   with TMA, overwrites each row with R_n phi(q_n) (bf16) while taking
-//   den = phi(q_n) . z_<=b + eps in fp32, runs num = Q~ S_<=b on tcgen05
-//   (M = 128 tokens, N = d, K = d), reads num back from TMEM, divides, and
-//   stores bf16 rows with a TMA store (or plain stores for a ragged tile).
+// Pass 1, partial_tc_kernel: one CTA per state chunk (<= 1024 tokens of one
+//   block of one head).  A producer warp streams 128-token K and V tiles into
+//   shared memory with TMA (64B/128B swizzle).  Four transform warps overwrite
+//   each K row in place with R_m phi(k_m) (bf16) and, for d = 32, also write
+//   phi(k_m) into a second tile.  One MMA thread accumulates
+//       [K~^T ; phi(K)^T] x [V | 1]      (tcgen05.mma, fp32 in TMEM)
+//   so the d x d block state P = K~^T V and the denominator state
+//   zp = sum phi(k) come out of one contraction; both operands are MN-major
+//   views of the token-major tiles.  For d = 64 the tensor core computes P and
+//   the transform warps sum zp in fp32 registers.  The transform warps then
+//   write the chunk's partial state; the last chunk of each head to finish
+//   (atomic counter, no waiting) runs the fixed-order inclusive scan over
+//   blocks for that head.
+// Pass 2, output_tc_kernel: one CTA per group of <= 8 query tiles of one block
+//   of one head.  Epilogue warps first turn S_<=b, z_<=b into a bf16 B operand
+//       [[S, 0], [0, z_hi z_lo]]   (K = 2d rows, N = d + 16 columns)
+//   A producer warp streams Q tiles; transform warps write [R phi(q) | phi(q)]
+//   as the bf16 A operand; one MMA thread computes
+//       [Q~ | phi(Q)] x B = [num | phi(q).z_hi | phi(q).z_lo]
+//   into one of two TMEM accumulators; epilogue warps read it back, form
+//   o = num / (phi(q).z + eps) in fp32, write bf16 rows in place over the Q
+//   tile and store them with TMA (plain stores for a ragged last tile).
 //
-// Warp roles: warps 0-3 own one token row each per tile (thread r <-> row r;
-// they also read TMEM lanes 32w..32w+31); warp 4 lane 0 issues the TMA loads.
-// Thread 0 issues MMAs.  All waits are bounded (see ptx::mbar_wait_bounded).
+// Roles hand tiles to each other through mbarriers only (no CTA-wide barrier
+// inside the main loops) and every wait is bounded (ptx::mbar_wait_bounded).
+// Grids are ordered chunk-index-major so the short last chunks run last.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -27,15 +36,6 @@
 namespace blin {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
-
-template <int D>
-struct TcCfg {
-    static constexpr int ROWB = D * 2;                  // bytes per token row (bf16)
-    static constexpr int TB = kTile * ROWB;             // bytes per 128-row tile
-    static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;  // 64B : 128B swizzle
-    static constexpr int P1_STAGES = D == 32 ? 4 : 3;
-    static constexpr int P2_STAGES = 4;
-};
 
 // Byte offset of 16-byte chunk `j` of row `r` inside a swizzled tile whose base
 // is 1024-byte aligned (64B swizzle: rows of 64 B; 128B swizzle: rows of 128 B).
@@ -50,6 +50,11 @@ __device__ __forceinline__ uint32_t swz_chunk(int r, int j) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Token position bookkeeping: relative frame t, row y, column x of a token,
@@ -71,34 +76,54 @@ struct TokPos {
     }
 };
 
+// Where a CTA reads RoPE (cos, sin) pairs from: its shared-memory copy (frame
+// window + full y and x tables) when the call's tables are small, else the
+// global table.
+struct RopeTab {
+    const float2 *t, *y, *x;  // t indexed by relative frame (window offset folded in)
+};
+
+// Fills this CTA's shared-memory copy of the call's RoPE table (the
+// tensor-core path is only chosen when it fits; transform threads only, a
+// barrier among them must follow).
+template <int PT, int PY, int PX>
+__device__ __forceinline__ RopeTab load_rope_tab(const KGeom &g, float2 *s_tab, int tid, int nthreads) {
+    const int n = g.T * PT + g.Hg * PY + g.Wg * PX;
+    for (int i = tid; i < n; i += nthreads) s_tab[i] = rope_entry(i, g.T, g.t0, g.Hg, PT, PY, PX, g.theta);
+    RopeTab r;
+    r.t = s_tab;
+    r.y = s_tab + g.tab_y;
+    r.x = s_tab + g.tab_x;
+    return r;
+}
+
 // phi (ReLU) then 3D RoPE of one token row held as D/2 bf16x2 words (pair p =
-// features 2p, 2p+1, low half = even feature).  Optionally accumulates the
-// unrotated phi into zp and the unrotated phi . z into den.
-// (RoPE inside linear attention: talk transcript; RoPE only in the numerator,
-// phi . z without RoPE in the denominator: news article, positional encoding.)
-template <int D, int PT, int PY, int PX, bool ZP, bool DEN>
-__device__ __forceinline__ void phi_rope_row(uint32_t (&w)[D / 2], const KGeom &g, const TokPos &tp,
-                                             float (&zp)[D], float &den, const float *zs) {
+// features 2p, 2p+1, low half = even feature).  Writes phi into `ph` (bf16x2,
+// exact) and optionally sums phi into zp.
+// (RoPE inside linear attention: talk transcript; RoPE only in the numerator:
+// news article, positional-encoding paragraph.)
+template <int D, int PT, int PY, int PX, bool ZP>
+__device__ __forceinline__ void phi_rope_row(uint32_t (&w)[D / 2], uint32_t (&ph)[D / 2], const RopeTab &tab,
+                                             const TokPos &tp, float *zp) {
     static_assert(PT + PY + PX == D / 2, "split must cover d");
-    const float2 *rt = g.tab + tp.t * PT;
-    const float2 *ry = g.tab + g.tab_y + tp.y * PY;
-    const float2 *rx = g.tab + g.tab_x + tp.x * PX;
+    const float2 *rt = tab.t + tp.t * PT;
+    const float2 *ry = tab.y + tp.y * PY;
+    const float2 *rx = tab.x + tp.x * PX;
 #pragma unroll
     for (int p = 0; p < D / 2; ++p) {
-        const float2 cs = p < PT ? __ldg(rt + p) : (p < PT + PY ? __ldg(ry + (p - PT)) : __ldg(rx + (p - PT - PY)));
-        const float a = fmaxf(__uint_as_float(w[p] << 16), 0.f);
-        const float b = fmaxf(__uint_as_float(w[p] & 0xFFFF0000u), 0.f);
+        const float2 cs = p < PT ? rt[p] : (p < PT + PY ? ry[p - PT] : rx[p - PT - PY]);
+        // ReLU on the packed pair (exact), then widen
+        __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162 *>(&w[p]);
+        hv = __hmax2(hv, __float2bfloat162_rn(0.f));
+        const uint32_t u = *reinterpret_cast<uint32_t *>(&hv);
+        ph[p] = u;
+        const float a = __uint_as_float(u << 16);
+        const float b = __uint_as_float(u & 0xFFFF0000u);
         if constexpr (ZP) {
             zp[2 * p] += a;
             zp[2 * p + 1] += b;
         }
-        if constexpr (DEN) {
-            den = fmaf(a, zs[2 * p], den);
-            den = fmaf(b, zs[2 * p + 1], den);
-        }
-        const float ra = fmaf(a, cs.x, -b * cs.y);
-        const float rb = fmaf(a, cs.y, b * cs.x);
-        w[p] = pack_bf16x2(ra, rb);
+        w[p] = pack_bf16x2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
     }
 }
 
@@ -127,219 +152,494 @@ __device__ __forceinline__ void zero_row(uint8_t *tile, int r) {
         *reinterpret_cast<uint4 *>(tile + swz_chunk<D>(r, j)) = make_uint4(0, 0, 0, 0);
 }
 
+// Rounds a pointer into the kernel's dynamic shared memory up to 1024 bytes by
+// indexing from it (not through an integer cast), so the compiler keeps every
+// derived access in the shared address space (LDS/STS, not generic loads).
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+    const uint32_t a = ptx::smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-template <int D>
-constexpr int partial_tc_smem_bytes() {
-    return TcCfg<D>::P1_STAGES * 2 * TcCfg<D>::TB + 1024 + 256;
-}
-template <int D>
-constexpr int output_tc_smem_bytes() {
-    return TcCfg<D>::P2_STAGES * TcCfg<D>::TB + D * TcCfg<D>::ROWB + D * 4 + 1024 + 256;
+// Loads `n` (1, 2 or 32) consecutive fp32 TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld_2cols(uint32_t taddr, float &a, float &b) {
+    uint32_t r0, r1;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0), "=r"(r1)
+        : "r"(taddr)
+        : "memory");
+    a = __uint_as_float(r0);
+    b = __uint_as_float(r1);
 }
 
-// =========================================================================== pass 1
+// ---------------------------------------------------------------------------- output B operand
+template <int D>
+struct OutB {  // the output kernel's B operand: K atoms of N rows, bf16, K-major, swizzled
+    static constexpr int N = D + 16;          // num | phi.z_hi | phi.z_lo | zero pad
+    static constexpr int ROWB = 2 * D;
+    static constexpr int BATOM = N * ROWB;    // one K atom
+    static constexpr int IMG = 2 * BATOM;     // atom 0: S part, atom 1: z part
+};
+
+template <int D>
+__device__ __forceinline__ int swz_bits(int n) {
+    return D == 32 ? ((n >> 1) & 3) : (n & 7);
+}
+
+// One 16-byte chunk (`item`, in storage order) of the B operand built from the
+// fp32 prefix state `pre` (S row-major [key feature][value feature], then z):
+// atom 0 row n < D holds S[.][n]; atom 1 rows D and D+1 hold z split into a
+// bf16 high part and the bf16 rounding of the remainder; all else is zero.
+template <int D>
+__device__ __forceinline__ uint4 b_operand_chunk(const float *pre, int item) {
+    using B = OutB<D>;
+    const int atom = item / (B::BATOM / 16), rr = item % (B::BATOM / 16);
+    const int n = rr / (D / 8), gq = (rr % (D / 8)) ^ swz_bits<D>(n);
+    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+    if (atom == 0 && n < D) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) w4[u] = pack_bf16x2(pre[(8 * gq + 2 * u) * D + n], pre[(8 * gq + 2 * u + 1) * D + n]);
+    } else if (atom == 1 && (n == D || n == D + 1)) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float zz[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float z = pre[D * D + 8 * gq + 2 * u + h];
+                const float hi = __bfloat162float(__float2bfloat16_rn(z));
+                zz[h] = n == D ? hi : z - hi;
+            }
+            w4[u] = pack_bf16x2(zz[0], zz[1]);
+        }
+    }
+    return make_uint4(w4[0], w4[1], w4[2], w4[3]);
+}
+
+// ============================================================================ shared control
+__device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
+
+// Tiles of a work unit alternate between two transform groups (tile k goes to
+// group k & 1).  A group's first tile of a unit is tile 0 or 1; it then steps
+// by two tiles.  The producer ends the stream with two markers: -1 (passed on
+// through the operand ring) for the group that sees the end first, -2 for the
+// other group, which just stops.
+constexpr int kEndFirst = -1, kEndSecond = -2;
+
+// ============================================================================ pass 1
+template <int D>
+struct P1 {
+    static constexpr int ROWB = 2 * D;
+    static constexpr int TB = kTile * ROWB;
+    static constexpr int M = D == 32 ? 64 : 128;          // [K~^T ; phi(K)^T]
+    static constexpr int N = D == 32 ? D + 8 : D + 16;   // [V | ones]
+    static constexpr int NL = D == 32 ? 7 : 2;           // landing stages: K | V (TMA)
+    static constexpr int NO = D == 32 ? 3 : 2;           // operand sets: K~ | phi | V
+    static constexpr int NACC = 4;                       // TMEM accumulators (chunks in flight)
+    static constexpr int ACOLS = D == 32 ? 64 : 128;     // TMEM columns per accumulator
+    static constexpr uint32_t TCOLS = NACC * ACOLS;
+    static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
+    static constexpr int CTRL = 1024;
+    static constexpr int FIXED = NL * 2 * TB + NO * 3 * TB + TB + CTRL + 1024;  // + RoPE table
+    static constexpr int THREADS = 448;  // warps 0-7 transform, 8-11 epilogue, 12 producer, 13 MMA
+};
+
+// Persistent, one CTA per SM: CTA j takes chunks j, j + grid, ... (chunk-index
+// major, so the short last chunk of every block comes last and spreads evenly).  TMA lands K and V tiles in a deep ring; transform warps
+// release each landing slot as soon as they have read it and write the MMA
+// operands (K~, phi(K), V) into a second ring, so DRAM latency is covered by
+// the landing ring alone.  Four TMEM accumulators let chunk epilogues
+// (TMEM -> chunk partial in global memory) trail the MMAs.
 template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(448, 1)
     partial_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                       KGeom g, int *watchdog) {
-    using C = TcCfg<D>;
-    constexpr int NS = C::P1_STAGES;
-    constexpr int TB = C::TB, ROWB = C::ROWB;
-    constexpr uint32_t IDESC = ptx::idesc_bf16_f32(64, D, 1, 1);
-    constexpr uint32_t TCOLS = D;  // 64 x D fp32 accumulator (M = 64 layout: lanes 0-15 of each subpartition)
+    using C = P1<D>;
+    constexpr int NL = C::NL, NO = C::NO, TB = C::TB, ROWB = C::ROWB, E = D * D + D;
+    constexpr uint32_t IDESC = ptx::idesc_bf16_f32(C::M, C::N, 1, 1);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NS * 2 * TB);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * NS + 1);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    auto ktile = [&](int s) { return smem + s * 2 * TB; };
-    auto vtile = [&](int s) { return smem + s * 2 * TB + TB; };
-    auto full = [&](int s) { return ptx::smem_u32(bars + s); };
-    auto empty = [&](int s) { return ptx::smem_u32(bars + NS + s); };
-    const uint32_t accbar = ptx::smem_u32(bars + 2 * NS);
+    uint8_t *land = smem;                       // [NL][K | V]
+    uint8_t *opnd = land + NL * 2 * TB;         // [NO][K~ | phi | V]
+    uint8_t *ones = opnd + NO * 3 * TB;         // constant B block
+    uint8_t *ctrl = ones + TB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
+    int *linfo = reinterpret_cast<int *>(ctrl + 256);                 // [NL][4] unit, tile, valid, last
+    int *oinfo = linfo + 4 * NL;                                      // [NO][4]
+    int *acc_unit = oinfo + 4 * NO;                                   // [NACC]
+    volatile int *flags = reinterpret_cast<volatile int *>(acc_unit + C::NACC);  // abort, epilogue
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_unit + C::NACC + 4);
+    float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
+    auto lk = [&](int s) { return land + s * 2 * TB; };
+    auto lv = [&](int s) { return land + s * 2 * TB + TB; };
+    auto ok_ = [&](int s) { return opnd + s * 3 * TB; };
+    auto op_ = [&](int s) { return opnd + s * 3 * TB + TB; };
+    auto ov_ = [&](int s) { return opnd + s * 3 * TB + 2 * TB; };
+    auto lfull = [&](int s) { return ptx::smem_u32(bars + s); };
+    auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
+    auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
+    auto oempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
+    constexpr int NA = C::NACC;
+    auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + a); };
+    auto accp = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + NA + a); };
+    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 2 * NA + a); };
 
-    const int c = blockIdx.x, b = blockIdx.y, bh = blockIdx.z;
-    const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
-    const int btok0 = fb * g.HW, bntok = (fe - fb) * g.HW;
-    const int cs = c * kChunk;
-    if (cs >= bntok) return;  // CTA-uniform, before any barrier or TMEM use
-    const int clen = min(kChunk, bntok - cs);
-    const int ntiles = (clen + kTile - 1) / kTile;
-    const int row0 = bh * g.N + btok0 + cs;
+    const int units = g.cpb * g.nblk * g.BH;
+    const int per_c = g.nblk * g.BH;
+    // chunk-index-major order: the short last chunks of every block come last
+    auto decode = [&](int u, int &bh, int &b, int &c) {
+        c = u / per_c;
+        const int rem = u - c * per_c;
+        bh = rem / g.nblk;
+        b = rem - bh * g.nblk;
+    };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) {
-            ptx::mbar_init(full(s), 1);
-            ptx::mbar_init(empty(s), 1);
+        for (int s = 0; s < NL; ++s) {
+            ptx::mbar_init(lfull(s), 1);
+            ptx::mbar_init(lempty(s), 128);
         }
-        ptx::mbar_init(accbar, 1);
-        *abort_flag = 0;
+        for (int s = 0; s < NO; ++s) {
+            ptx::mbar_init(ofull(s), 128);
+            ptx::mbar_init(oempty(s), 1);
+        }
+        for (int a = 0; a < NA; ++a) {
+            ptx::mbar_init(accf(a), 1);
+            ptx::mbar_init(accp(a), 1);
+            ptx::mbar_init(acce(a), 128);
+        }
+        flags[0] = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TCOLS);
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TCOLS);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    if (tid == 0) griddep_launch_dependents();
 
-    if (warp == 4) {
+    if (warp == 12) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ptx::tma_prefetch_map(&mk);
             ptx::tma_prefetch_map(&mv);
-            for (int i = 0; i < ntiles; ++i) {
-                const int s = i % NS;
-                // on timeout just stop issuing: the compute warps then time out on
-                // `full` themselves and agree on the abort across their barrier
-                if (i >= NS &&
-                    !ptx::mbar_wait_bounded(empty(s), ((i / NS) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
-                                            kWaitLimitNs))
-                    break;
-                ptx::mbar_arrive_expect_tx(full(s), 2 * TB);
-                ptx::tma_load_2d(ptx::smem_u32(ktile(s)), &mk, full(s), 0, row0 + i * kTile);
-                ptx::tma_load_2d(ptx::smem_u32(vtile(s)), &mv, full(s), 0, row0 + i * kTile);
-            }
-        }
-    } else {
-        const int r = tid;  // token row owned by this thread
-        TokPos tp;
-        tp.init(g, btok0 + cs + r);
-        const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
-        float zp[D];
-#pragma unroll
-        for (int i = 0; i < D; ++i) zp[i] = 0.f;
-        float unused_den = 0.f;
-        bool ok = true;
-        for (int i = 0; i < ntiles; ++i) {
-            const int s = i % NS;
-            ok = ptx::mbar_wait_bounded(full(s), (i / NS) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs);
-            if (!ok) *abort_flag = 1;
-            if (ok) {
-                if (i * kTile + r < clen) {
-                    uint32_t w[D / 2];
-                    load_row<D>(ktile(s), r, w);
-                    phi_rope_row<D, PT, PY, PX, true, false>(w, g, tp, zp, unused_den, nullptr);
-                    store_row<D>(ktile(s), r, w);
-                } else {
-                    // rows past the chunk: zero both operands so they add nothing
-                    zero_row<D>(ktile(s), r);
-                    zero_row<D>(vtile(s), r);
-                }
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(1, 128);
-            if (*abort_flag) { ok = false; break; }
-            if (r == 0) {
-                ptx::tc_fence_after_sync();
-                const uint32_t ka = ptx::smem_u32(ktile(s)), va = ptx::smem_u32(vtile(s));
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    // A = K~^T: MN-major, 8-token groups every 8 rows; for d = 32 the
-                    // second 32-row M atom (rows 32..63, unused) is the V tile at +TB.
-                    const uint64_t ad = ptx::smem_desc(ka + kk * 16 * ROWB, TB, 8 * ROWB, C::LAYOUT);
-                    const uint64_t bd = ptx::smem_desc(va + kk * 16 * ROWB, TB, 8 * ROWB, C::LAYOUT);
-                    ptx::mma_bf16_ss(tmem, ad, bd, IDESC, (i > 0 || kk > 0) ? 1u : 0u);
-                }
-                ptx::mma_commit(empty(s));
-                if (i == ntiles - 1) ptx::mma_commit(accbar);
-            }
-            tp.advance(g, dx, dy, dt);
-        }
-        // ---- epilogue: P from TMEM, zp via a fixed-order shared-memory reduction
-        float *out = g.part + ((size_t)(bh * g.nblk + b) * g.cpb + c) * (D * D + D);
-        if (ok) ok = ptx::mbar_wait_bounded(accbar, 0, watchdog, WD_PARTIAL_ACC, kWaitLimitNs);
-        ptx::tc_fence_after_sync();
-        {
-            // M = 64 accumulator: row m lives in TMEM lane (m % 16) + 32 * (m / 16).
-            // tcgen05.ld is warp-collective, so only the store depends on `ok`.
-            const int m = 16 * warp + lane;
-            if (D == 64 || warp < 2) {
-#pragma unroll
-                for (int half = 0; half < D / 32; ++half) {
-                    float v[32];
-                    ptx::tmem_ld_32cols(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * half, v);
-                    if (ok && lane < 16) {
-                        float4 *dst = reinterpret_cast<float4 *>(out + m * D + 32 * half);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            int k = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {  // static round robin
+                int bh, b, c;
+                decode(u, bh, b, c);
+                const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
+                const int bntok = (fe - fb) * g.HW, cs = c * kChunk;
+                if (cs < bntok) {
+                    const int clen = min(kChunk, bntok - cs), ntiles = (clen + kTile - 1) / kTile;
+                    const int row0 = bh * g.N + fb * g.HW + cs;
+                    for (int t = 0; t < ntiles; ++t, ++k) {
+                        const int sl = k % NL;
+                        if (k >= NL && !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog,
+                                                               WD_PARTIAL_EMPTY, kWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        int *inf = linfo + 4 * sl;
+                        inf[0] = u;
+                        inf[1] = t;
+                        inf[2] = min(kTile, clen - t * kTile);
+                        inf[3] = t == ntiles - 1;
+                        ptx::mbar_arrive_expect_tx(lfull(sl), 2 * TB);
+                        ptx::tma_load_2d(ptx::smem_u32(lk(sl)), &mk, lfull(sl), 0, row0 + t * kTile);
+                        ptx::tma_load_2d(ptx::smem_u32(lv(sl)), &mv, lfull(sl), 0, row0 + t * kTile);
                     }
                 }
             }
+            for (int e = 0; ok && e < 2; ++e, ++k) {  // end markers, one per transform group
+                const int sl = k % NL;
+                if (k >= NL && !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
+                                                       kWaitLimitNs))
+                    break;
+                linfo[4 * sl] = e == 0 ? kEndFirst : kEndSecond;
+                ptx::mbar_arrive(lfull(sl));
+            }
         }
-        ptx::tc_fence_before_sync();
-        ptx::named_bar_sync(1, 128);
-        // stage memory is idle now (all loads consumed, all MMAs complete)
-        float *red = reinterpret_cast<float *>(smem);
+    } else if (warp == 13) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int nu = 0;
+            bool ok = true;
+            for (int k = 0;; ++k) {
+                const int so = k % NO;
+                if (flags[0] ||
+                    !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                const int *inf = oinfo + 4 * so;
+                const int u = ld_volatile(inf), t = ld_volatile(inf + 1), last = ld_volatile(inf + 3);
+                if (u < 0) break;
+                const int a = nu % NA;
+                if (t == 0 && nu >= NA &&
+                    !ptx::mbar_wait_bounded(acce(a), ((nu / NA) - 1) & 1, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after_sync();
+                const uint32_t ka = ptx::smem_u32(ok_(so)), va = ptx::smem_u32(ov_(so));
+                const uint32_t lbo_b = ptx::smem_u32(ones) - va;  // N atom 1 = the ones block
 #pragma unroll
-        for (int i = 0; i < D; ++i) red[r * (D + 1) + i] = zp[i];
-        ptx::named_bar_sync(1, 128);
-        if (ok && r < D) {
-            float s = 0.f;
-            for (int t = 0; t < kTile; ++t) s += red[t * (D + 1) + r];
-            out[D * D + r] = s;
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones
+                    const uint64_t ad = ptx::smem_desc(ka + kk * 16 * ROWB, TB, 8 * ROWB, C::LAYOUT);
+                    const uint64_t bd = ptx::smem_desc(va + kk * 16 * ROWB, lbo_b, 8 * ROWB, C::LAYOUT);
+                    ptx::mma_bf16_ss(tmem + a * C::ACOLS, ad, bd, IDESC, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::mma_commit(oempty(so));
+                if (last) {
+                    acc_unit[a] = u;
+                    ptx::mbar_arrive(accp(a));
+                    ptx::mma_commit(accf(a));
+                    ++nu;
+                }
+            }
+            if (!ok) flags[0] = 1;
+            const int a = nu % NA;  // tell the epilogue there is nothing more
+            if (ok && (nu < NA || ptx::mbar_wait_bounded(acce(a), ((nu / NA) - 1) & 1, watchdog, WD_PARTIAL_ACC,
+                                                         kWaitLimitNs))) {
+                acc_unit[a] = -1;
+                ptx::mbar_arrive(accp(a));
+            }
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ transform warps (two groups)
+        const int grp = warp >> 2, r = tid & 127;
+        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 256);
+        {
+            uint4 *o4 = reinterpret_cast<uint4 *>(ones);  // all 1.0, so its swizzle is irrelevant
+            for (int i = tid; i < TB / 16; i += 256) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        }
+        ptx::named_bar_sync(1, 256);
+        const int step = 2 * kTile;
+        const int dx = step % g.Wg, dy = (step / g.Wg) % g.Hg, dt = step / g.HW;
+        TokPos tp{0, 0, 0};
+        for (int k = grp;; k += 2) {
+            const int sl = k % NL, so = k % NO;
+            if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            const int *inf = linfo + 4 * sl;
+            const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
+            const int last = ld_volatile(inf + 3);
+            if (u == kEndSecond) break;
+            // read this row of the landed tiles and give the slot back right away
+            uint32_t w[D / 2], vw[D / 2], ph[D / 2];
+            const bool live = u >= 0 && r < valid;
+            if (live) {
+                load_row<D>(lk(sl), r, w);
+                load_row<D>(lv(sl), r, vw);
+            }
+            if (u >= 0) ptx::mbar_arrive(lempty(sl));
+            if (k >= NO &&
+                !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            if (u == kEndFirst) {  // pass the end on to the MMA issuer, in operand order
+                if (r == 0) oinfo[4 * so] = kEndFirst;
+                ptx::mbar_arrive(ofull(so));
+                break;
+            }
+            if (t <= 1) {
+                int bh, b, c;
+                decode(u, bh, b, c);
+                tp.init(g, block_frame_begin(g, b) * g.HW + c * kChunk + t * kTile + r);
+            } else {
+                tp.advance(g, dx, dy, dt);
+            }
+            if (live) {
+                phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
+                store_row<D>(ok_(so), r, w);
+                store_row<D>(op_(so), r, ph);
+                store_row<D>(ov_(so), r, vw);
+            } else {  // rows past the chunk add nothing
+                zero_row<D>(ok_(so), r);
+                zero_row<D>(op_(so), r);
+                zero_row<D>(ov_(so), r);
+            }
+            ptx::fence_proxy_async_smem();
+            if (r == 0) {
+                int *oi = oinfo + 4 * so;
+                oi[0] = u;
+                oi[1] = t;
+                oi[2] = valid;
+                oi[3] = last;
+            }
+            ptx::mbar_arrive(ofull(so));
+        }
+    } else if (warp < 12) {
+        // ------------------------------------------------------------ epilogue warps (8-11)
+        const int er = tid - 256, sub = warp & 3;
+        // M = 64 (d = 32): accumulator row m in TMEM lane (m % 16) + 32 * (m / 16);
+        // M = 128 (d = 64): row m in lane m.  Rows [0, D) hold P, rows [D, 2D) hold
+        // phi^T against the ones block, i.e. zp, in column D.
+        constexpr int RPS = D == 32 ? 16 : 32;  // accumulator rows per TMEM subpartition
+        for (int nu = 0;; ++nu) {
+            const int a = nu % NA, ph = (nu / NA) & 1;
+            if (er == 0) {  // one thread waits and decides for all 128 (named barrier below)
+                int u = -1;
+                if (!flags[0] && ptx::mbar_wait_bounded(accp(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
+                    u = ld_volatile(acc_unit + a);
+                    if (u >= 0 && !ptx::mbar_wait_bounded(accf(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
+                        u = -1;
+                        flags[0] = 1;
+                    }
+                } else {
+                    flags[0] = 1;
+                }
+                flags[1] = u;
+            }
+            ptx::named_bar_sync(2, 128);
+            const int u = flags[1];
+            ptx::named_bar_sync(2, 128);  // everyone has read flags[1] before it is rewritten
+            if (u < 0) break;
+            ptx::tc_fence_after_sync();
+            int bh, b, c;
+            decode(u, bh, b, c);
+            float *out = g.part + ((size_t)(bh * g.nblk + b) * g.cpb + c) * E;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
+            if (sub < 2) {
+                const int m = RPS * sub + lane;  // P row
+#pragma unroll
+                for (int half = 0; half < D / 32; ++half) {
+                    float v[32];
+                    ptx::tmem_ld_32cols(taddr + 32 * half, v);
+                    if (lane < RPS) {
+                        float4 *dst = reinterpret_cast<float4 *>(out + m * D + 32 * half);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    }
+                }
+            } else {
+                float zv, unused;
+                tmem_ld_2cols(taddr + D, zv, unused);
+                if (lane < RPS) out[D * D + RPS * (sub - 2) + lane] = zv;
+            }
+            ptx::tc_fence_before_sync();
+            ptx::mbar_arrive(acce(a));  // accumulator a is free again
         }
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem, TCOLS);
+        ptx::tmem_dealloc(tmem, C::TCOLS);
     }
 }
 
-// =========================================================================== pass 2
+// ============================================================================ pass 2
+template <int D>
+struct P2 {
+    static constexpr int ROWB = 2 * D;
+    static constexpr int TB = kTile * ROWB;
+    static constexpr int NL = D == 32 ? 12 : 2;        // landing stages (Q tiles)
+    static constexpr int NO = D == 32 ? 3 : 2;         // operand sets: q~ | phi(q)
+    static constexpr int NSTG = D == 32 ? 2 : 1;       // O staging buffers per epilogue group
+    static constexpr int N = OutB<D>::N;               // num | phi.z_hi | phi.z_lo | pad
+    static constexpr int BATOM = OutB<D>::BATOM;       // one K atom of B (N rows)
+    static constexpr int IMG = OutB<D>::IMG;
+    static constexpr int ACOLS = D == 32 ? 64 : 128;   // TMEM columns per accumulator
+    static constexpr uint32_t TCOLS = 2 * ACOLS;
+    static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
+    static constexpr int PRE = (D * D + D) * 4;        // one fp32 prefix state (S, z)
+    static constexpr int NBARS = 2 * NL + 2 * NO + 12;
+    static constexpr int INFO = (NBARS * 8 + 15) / 16 * 16;
+    static constexpr int CTRL = 1024;
+    static constexpr int FIXED = NL * TB + NO * 2 * TB + 2 * NSTG * TB + 2 * IMG + 2 * PRE + CTRL + 1024;  // + table
+    static constexpr int THREADS = 608;  // warps 0-7 transform, 8-15 epilogue, 16 producer, 17 MMA, 18 B prep
+    static_assert(INFO + 32 * NL + 32 * NO + 32 + 64 + 16 <= CTRL, "control block overflow");
+};
+
+// Persistent, one CTA per SM: CTA j takes groups j, j + grid, ... of <= 8 query
+// tiles of one (head, block).  Per group the
+// producer bulk-copies the fp32 prefix state, which a B-prep warp turns into
+// the bf16 B operand (both double-buffered); per tile it lands Q in a deep ring.  Two transform groups write [R phi(q) | phi(q)] into
+// an operand ring; the MMA issuer alternates two TMEM accumulators, and
+// epilogue group e (warps 8+4e..11+4e) owns accumulator e: it divides, writes
+// bf16 rows to its staging buffer and stores them with TMA (plain stores for a
+// ragged tile).
 template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(608, 1)
     output_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo,
                      KGeom g, __nv_bfloat16 *o, int *watchdog) {
-    using C = TcCfg<D>;
-    constexpr int NS = C::P2_STAGES;
-    constexpr int TB = C::TB, ROWB = C::ROWB;
-    constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, D, 0, 0);
-    constexpr uint32_t TCOLS = 2 * D;  // two 128 x D fp32 accumulators
+    using C = P2<D>;
+    constexpr int NL = C::NL, NO = C::NO, NSTG = C::NSTG, TB = C::TB, ROWB = C::ROWB;
+    constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, C::N, 0, 0);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *sop = smem + NS * TB;  // S_<=b as bf16, K-major B operand: row n = value feature j
-    float *zs = reinterpret_cast<float *>(sop + D * ROWB);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(zs + D);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * NS + 2);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    auto qtile = [&](int s) { return smem + s * TB; };
-    auto full = [&](int s) { return ptx::smem_u32(bars + s); };
-    auto empty = [&](int s) { return ptx::smem_u32(bars + NS + s); };
-    auto mmad = [&](int a) { return ptx::smem_u32(bars + 2 * NS + a); };
+    uint8_t *land = smem;                        // [NL][Q]
+    uint8_t *opnd = land + NL * TB;              // [NO][q~ | phi]
+    uint8_t *stg = opnd + NO * 2 * TB;           // [2 groups][NSTG][O]
+    uint8_t *bbuf = stg + 2 * NSTG * TB;         // [2][IMG] bf16 B operand
+    uint8_t *pbuf = bbuf + 2 * C::IMG;           // [2][PRE] fp32 prefix state
+    uint8_t *ctrl = pbuf + 2 * C::PRE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
+    int *linfo = reinterpret_cast<int *>(ctrl + C::INFO);  // [NL][8]: unit, tile, valid, ord, row0, last
+    int *oinfo = linfo + 8 * NL;                          // [NO][8]
+    int *ainfo = oinfo + 8 * NO;                          // [2][4]: valid (-1 = end), row0
+    volatile int *flags = reinterpret_cast<volatile int *>(ainfo + 8);  // [0] abort, [2..3] prefix slots, [4+4e..]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ainfo + 8 + 16);
+    float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
+    auto lq = [&](int s) { return land + s * TB; };
+    auto oq = [&](int s) { return opnd + s * 2 * TB; };
+    auto oph = [&](int s) { return opnd + s * 2 * TB + TB; };
+    auto lfull = [&](int s) { return ptx::smem_u32(bars + s); };
+    auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
+    auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
+    auto oempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
+    auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + a); };
+    auto accp = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 2 + a); };
+    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 4 + a); };
+    auto bfull = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 6 + a); };
+    auto bempty = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 8 + a); };
+    auto pfull = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 10 + a); };
 
-    const int c = blockIdx.x, b = blockIdx.y, bh = blockIdx.z;
-    const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
-    const int btok0 = fb * g.HW, bntok = (fe - fb) * g.HW;
-    const int qs = c * kQTiles * kTile;
-    if (qs >= bntok) return;  // CTA-uniform
-    const int qlen = min(kQTiles * kTile, bntok - qs);
-    const int ntiles = (qlen + kTile - 1) / kTile;
-    const int row0 = bh * g.N + btok0 + qs;
+    const int units = g.qcpb * g.nblk * g.BH;
+    const int per_q = g.nblk * g.BH;
+    auto decode = [&](int u, int &bh, int &b, int &qc) {
+        qc = u / per_q;
+        const int rem = u - qc * per_q;
+        bh = rem / g.nblk;
+        b = rem - bh * g.nblk;
+    };
+    constexpr int QG = kQTiles * kTile;  // tokens per group
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) {
-            ptx::mbar_init(full(s), 1);
-            ptx::mbar_init(empty(s), 1);
+        for (int s = 0; s < NL; ++s) {
+            ptx::mbar_init(lfull(s), 1);
+            ptx::mbar_init(lempty(s), 128);
         }
-        ptx::mbar_init(mmad(0), 1);
-        ptx::mbar_init(mmad(1), 1);
-        *abort_flag = 0;
+        for (int s = 0; s < NO; ++s) {
+            ptx::mbar_init(ofull(s), 128);
+            ptx::mbar_init(oempty(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(accf(a), 1);
+            ptx::mbar_init(accp(a), 1);
+            ptx::mbar_init(acce(a), 128);
+            ptx::mbar_init(bfull(a), 1);
+            ptx::mbar_init(bempty(a), 1);
+            ptx::mbar_init(pfull(a), 1);
+        }
+        flags[0] = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TCOLS);
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TCOLS);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before_sync();
@@ -347,119 +647,275 @@ __global__ void __launch_bounds__(160, 1)
     ptx::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 16) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ptx::tma_prefetch_map(&mq);
             ptx::tma_prefetch_map(&mo);
-            for (int i = 0; i < ntiles; ++i) {
-                const int s = i % NS;
-                if (i >= NS &&
-                    !ptx::mbar_wait_bounded(empty(s), ((i / NS) - 1) & 1, watchdog, WD_OUT_EMPTY,
-                                            kWaitLimitNs))
-                    break;
-                ptx::mbar_arrive_expect_tx(full(s), TB);
-                ptx::tma_load_2d(ptx::smem_u32(qtile(s)), &mq, full(s), 0, row0 + i * kTile);
+            int k = 0, nu = 0;
+            bool waited = false, ok = true;
+            auto issue_b = [&](int bh, int b, int ord) {
+                const int sl = ord & 1;
+                if (ord >= 2 &&
+                    !ptx::mbar_wait_bounded(bempty(sl), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))
+                    return false;
+                if (!waited) {  // the prefix states are written by the scan
+                    griddep_wait();
+                    waited = true;
+                }
+                flags[2 + sl] = 1;
+                ptx::mbar_arrive_expect_tx(pfull(sl), C::PRE);
+                ptx::bulk_load(ptx::smem_u32(pbuf + sl * C::PRE), g.prefix + ((size_t)bh * g.nblk + b) * (D * D + D),
+                               C::PRE, pfull(sl));
+                return true;
+            };
+            for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {  // static round robin
+                int bh, b, qc;
+                decode(u, bh, b, qc);
+                const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
+                const int bntok = (fe - fb) * g.HW, qs = qc * QG;
+                if (qs < bntok) {
+                    const int qlen = min(QG, bntok - qs), ntiles = (qlen + kTile - 1) / kTile;
+                    const int row0 = bh * g.N + fb * g.HW + qs;
+                    // first group: its Q tiles go out before waiting on pass 1
+                    const int early = waited ? 0 : min(ntiles, NL);
+                    if (early == 0 && !(ok = issue_b(bh, b, nu))) break;
+                    for (int t = 0; t < ntiles; ++t, ++k) {
+                        const int sl = k % NL;
+                        if (k >= NL &&
+                            !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY, kWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        int *inf = linfo + 8 * sl;
+                        inf[0] = u;
+                        inf[1] = t;
+                        inf[2] = min(kTile, qlen - t * kTile);
+                        inf[3] = nu;
+                        inf[4] = row0 + t * kTile;
+                        inf[5] = t == ntiles - 1;
+                        ptx::mbar_arrive_expect_tx(lfull(sl), TB);
+                        ptx::tma_load_2d(ptx::smem_u32(lq(sl)), &mq, lfull(sl), 0, row0 + t * kTile);
+                        if (early > 0 && t == early - 1 && !(ok = issue_b(bh, b, nu))) break;
+                    }
+                    ++nu;
+                }
             }
+            for (int e = 0; ok && e < 2; ++e, ++k) {  // end markers, one per transform group
+                const int sl = k % NL;
+                if (k >= NL &&
+                    !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY, kWaitLimitNs))
+                    break;
+                linfo[8 * sl] = e == 0 ? kEndFirst : kEndSecond;
+                ptx::mbar_arrive(lfull(sl));
+            }
+            // end marker for the B-prep warp
+            const int sl = nu & 1;
+            if (ok && (nu < 2 || ptx::mbar_wait_bounded(bempty(sl), ((nu >> 1) - 1) & 1, watchdog, WD_OUT_BREADY,
+                                                        kWaitLimitNs))) {
+                flags[2 + sl] = -1;
+                ptx::mbar_arrive(pfull(sl));
+            }
+        }
+    } else if (warp == 18) {
+        // ------------------------------------------------------------ B prep: fp32 prefix -> bf16 B operand
+        for (int ord = 0;; ++ord) {
+            const int sl = ord & 1;
+            if (flags[0] || !ptx::mbar_wait_bounded(pfull(sl), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            if (flags[2 + sl] < 0) break;
+            const float *pre = reinterpret_cast<const float *>(pbuf + sl * C::PRE);
+            uint4 *dst = reinterpret_cast<uint4 *>(bbuf + sl * C::IMG);
+            for (int item = lane; item < C::IMG / 16; item += 32) dst[item] = b_operand_chunk<D>(pre, item);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bfull(sl));
+        }
+    } else if (warp == 17) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            int k = 0;
+            for (;; ++k) {
+                const int so = k % NO, a = k & 1;
+                if (flags[0] || !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                const int *inf = oinfo + 8 * so;
+                const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
+                const int ord = ld_volatile(inf + 3), row0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
+                if (u < 0) break;
+                if ((k >= 2 &&
+                     !ptx::mbar_wait_bounded(acce(a), ((k >> 1) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs)) ||
+                    (t == 0 &&
+                     !ptx::mbar_wait_bounded(bfull(ord & 1), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after_sync();
+                const uint32_t qa = ptx::smem_u32(oq(so)), pa = ptx::smem_u32(oph(so));
+                const uint32_t ba = ptx::smem_u32(bbuf + (ord & 1) * C::IMG);
+#pragma unroll
+                for (int kk = 0; kk < 2 * D / 16; ++kk) {
+                    // K atom 0 = q~, K atom 1 = phi(q); +32 B per 16-element K step
+                    const int atom = kk / (D / 16), j = kk % (D / 16);
+                    const uint64_t ad = ptx::smem_desc((atom ? pa : qa) + 32 * j, 16, 8 * ROWB, C::LAYOUT);
+                    const uint64_t bd = ptx::smem_desc(ba + atom * C::BATOM + 32 * j, 16, 8 * ROWB, C::LAYOUT);
+                    ptx::mma_bf16_ss(tmem + a * C::ACOLS, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(oempty(so));
+                ainfo[4 * a] = valid;
+                ainfo[4 * a + 1] = row0;
+                ptx::mbar_arrive(accp(a));
+                ptx::mma_commit(accf(a));
+                if (last) ptx::mma_commit(bempty(ord & 1));
+            }
+            if (!ok) flags[0] = 1;
+            // tell both epilogue groups there is nothing more (tiles k and k + 1)
+            for (int j = 0; ok && j < 2; ++j) {
+                const int kk = k + j, a = kk & 1;
+                if (kk >= 2 &&
+                    !ptx::mbar_wait_bounded(acce(a), ((kk >> 1) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs))
+                    break;
+                ainfo[4 * a] = -1;
+                ptx::mbar_arrive(accp(a));
+            }
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ transform warps (two groups)
+        const int grp = warp >> 2, r = tid & 127;
+        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 256);
+        ptx::named_bar_sync(1, 256);
+        const int step = 2 * kTile;
+        const int dx = step % g.Wg, dy = (step / g.Wg) % g.Hg, dt = step / g.HW;
+        TokPos tp{0, 0, 0};
+        for (int k = grp;; k += 2) {
+            const int sl = k % NL, so = k % NO;
+            if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_OUT_FULL, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            const int *inf = linfo + 8 * sl;
+            const int u = ld_volatile(inf);
+            if (u == kEndSecond) break;
+            const int t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2), ord = ld_volatile(inf + 3);
+            const int row0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
+            uint32_t w[D / 2], ph[D / 2];
+            const bool live = u >= 0 && r < valid;
+            if (live) load_row<D>(lq(sl), r, w);
+            if (u >= 0) ptx::mbar_arrive(lempty(sl));  // landing slot read
+            if (k >= NO &&
+                !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            if (u == kEndFirst) {  // pass the end on to the MMA issuer, in operand order
+                if (r == 0) oinfo[8 * so] = kEndFirst;
+                ptx::mbar_arrive(ofull(so));
+                break;
+            }
+            if (t <= 1) {
+                int bh, b, qc;
+                decode(u, bh, b, qc);
+                tp.init(g, block_frame_begin(g, b) * g.HW + qc * QG + t * kTile + r);
+            } else {
+                tp.advance(g, dx, dy, dt);
+            }
+            if (live) {
+                phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
+                store_row<D>(oq(so), r, w);
+                store_row<D>(oph(so), r, ph);
+            } else {  // rows past the group: finite values, outputs not stored
+                zero_row<D>(oq(so), r);
+                zero_row<D>(oph(so), r);
+            }
+            ptx::fence_proxy_async_smem();
+            if (r == 0) {
+                int *oi = oinfo + 8 * so;
+                oi[0] = u;
+                oi[1] = t;
+                oi[2] = valid;
+                oi[3] = ord;
+                oi[4] = row0;
+                oi[5] = last;
+            }
+            ptx::mbar_arrive(ofull(so));
         }
     } else {
-        const int r = tid;
-        // ---- prologue: S_<=b (fp32, row i = key feature) -> bf16 B operand with
-        // row n = value feature j holding S[0..D)[j] (K-major, swizzled); z to smem.
-        const float *pre = g.prefix + ((size_t)bh * g.nblk + b) * (D * D + D);
-        for (int item = r; item < D * (D / 8); item += 128) {
-            const int j = item / (D / 8), gq = item % (D / 8);
-            uint32_t w4[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                w4[u] = pack_bf16x2(pre[(8 * gq + 2 * u) * D + j], pre[(8 * gq + 2 * u + 1) * D + j]);
-            *reinterpret_cast<uint4 *>(sop + swz_chunk<D>(j, gq)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-        if (r < D) zs[r] = pre[D * D + r];
-        ptx::fence_proxy_async_smem();
-        ptx::named_bar_sync(1, 128);
-
-        TokPos tp;
-        tp.init(g, btok0 + qs + r);
-        const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
-        float zp_unused[D];
-        const uint32_t sop_a = ptx::smem_u32(sop);
-        for (int i = 0; i < ntiles; ++i) {
-            const int s = i % NS, acc = i & 1;
-            bool ok = ptx::mbar_wait_bounded(full(s), (i / NS) & 1, watchdog, WD_OUT_FULL, kWaitLimitNs);
-            if (!ok) *abort_flag = 1;
-            const bool valid = ok && (i * kTile + r < qlen);
-            float den = 0.f;
-            if (valid) {
-                uint32_t w[D / 2];
-                load_row<D>(qtile(s), r, w);
-                phi_rope_row<D, PT, PY, PX, false, true>(w, g, tp, zp_unused, den, zs);
-                store_row<D>(qtile(s), r, w);
-            }
-            den += g.eps;
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(1, 128);
-            if (*abort_flag) break;
-            if (r == 0) {
-                ptx::tc_fence_after_sync();
-                const uint32_t qa = ptx::smem_u32(qtile(s));
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    // K-major: +32 B per 16-element K step inside the swizzled row
-                    const uint64_t ad = ptx::smem_desc(qa + kk * 32, 16, 8 * ROWB, C::LAYOUT);
-                    const uint64_t bd = ptx::smem_desc(sop_a + kk * 32, 16, 8 * ROWB, C::LAYOUT);
-                    ptx::mma_bf16_ss(tmem + acc * D, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+        // ------------------------------------------------------------ epilogue groups (warps 8-15)
+        const int e = (warp - 8) >> 2, sub = warp & 3, er = (tid - 256) & 127;
+        const int r = 32 * sub + lane;  // tile row read back by this thread (TMEM subpartition)
+        volatile int *gf = flags + 4 + 4 * e;
+        const uint32_t bar_id = 2 + e;
+        for (int n = 0;; ++n) {  // this group's n-th tile uses accumulator e
+            if (er == 0) {  // one thread waits and decides for the group (named barrier below)
+                int valid = -1;
+                if (!flags[0] && ptx::mbar_wait_bounded(accp(e), n & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
+                    valid = ld_volatile(ainfo + 4 * e);
+                    gf[1] = ld_volatile(ainfo + 4 * e + 1);
+                    if (valid >= 0 &&
+                        !ptx::mbar_wait_bounded(accf(e), n & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
+                        valid = -1;
+                        flags[0] = 1;
+                    }
+                } else {
+                    flags[0] = 1;
                 }
-                ptx::mma_commit(mmad(acc));
+                gf[0] = valid;
+                // the staging buffer about to be reused has been read by its TMA store
+                ptx::bulk_wait_group_read<NSTG - 1>();
             }
-            ok = ptx::mbar_wait_bounded(mmad(acc), (i >> 1) & 1, watchdog, WD_OUT_MMA, kWaitLimitNs);
-            if (!ok) *abort_flag = 1;
+            ptx::named_bar_sync(bar_id, 128);
+            const int valid = gf[0], trow0 = gf[1];
+            if (valid < 0) break;
             ptx::tc_fence_after_sync();
-            const bool full_tile = (i + 1) * kTile <= qlen;
-            const float inv = __frcp_rn(den);
-            {  // tcgen05.ld is warp-collective: executed by every lane, stores gated by `valid`
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + e * C::ACOLS;
+            float zh, zl;
+            tmem_ld_2cols(taddr + D, zh, zl);
+            const float inv = __frcp_rn(zh + zl + g.eps);
+            const bool full_tile = valid == kTile;
+            uint8_t *st = stg + (e * NSTG + (n % NSTG)) * TB;
 #pragma unroll
-                for (int half = 0; half < D / 32; ++half) {
-                    float v[32];
-                    ptx::tmem_ld_32cols(tmem + (static_cast<uint32_t>(32 * warp) << 16) + acc * D + 32 * half, v);
-                    uint32_t ow[16];
+            for (int half = 0; half < D / 32; ++half) {
+                float v[32];
+                ptx::tmem_ld_32cols(taddr + 32 * half, v);
+                uint32_t ow[16];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) ow[u] = pack_bf16x2(v[2 * u] * inv, v[2 * u + 1] * inv);
-                    if (valid && ok) {
-                        if (full_tile) {
+                for (int q = 0; q < 16; ++q) ow[q] = pack_bf16x2(v[2 * q] * inv, v[2 * q + 1] * inv);
+                if (r < valid) {
+                    if (full_tile) {
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                *reinterpret_cast<uint4 *>(qtile(s) + swz_chunk<D>(r, 4 * half + j)) =
-                                    make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
-                        } else {
-                            uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)row0 + i * kTile + r) * D + 32 * half);
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(st + swz_chunk<D>(r, 4 * half + j)) =
+                                make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)trow0 + r) * D + 32 * half);
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                dst[j] = make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
-                        }
+                        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
                     }
                 }
             }
             ptx::tc_fence_before_sync();
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(1, 128);
-            if (*abort_flag) break;
-            if (r == 0) {
-                if (full_tile) {
-                    ptx::tma_store_2d(&mo, ptx::smem_u32(qtile(s)), 0, row0 + i * kTile);
+            ptx::mbar_arrive(acce(e));  // accumulator e may be overwritten
+            if (full_tile) {
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(bar_id, 128);
+                if (er == 0) {
+                    ptx::tma_store_2d(&mo, ptx::smem_u32(st), 0, trow0);
                     ptx::bulk_commit_group();
-                    ptx::bulk_wait_group_read<0>();
                 }
-                ptx::mbar_arrive(empty(s));
             }
-            tp.advance(g, dx, dy, dt);
         }
-        if (r == 0) ptx::bulk_wait_group<0>();
+        if (er == 0) ptx::bulk_wait_group<0>();
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem, TCOLS);
+        ptx::tmem_dealloc(tmem, C::TCOLS);
     }
 }
 

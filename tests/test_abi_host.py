@@ -54,7 +54,8 @@ def ws(B, H, d, g):
 
 
 def test_workspace_size_formula():
-    # tables + partials + prefix states, each padded to 256 B, plus 256 B of alignment slack
+    # RoPE table + chunk partials + prefix states, each padded to 256 B, plus
+    # 256 B of alignment slack
     B, H, d = 1, 70, 32
     g = geom()
     E = d * d + d
