@@ -143,14 +143,25 @@ def dist_setup(ngpus: int):
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time (device clocks are per rank; the job is as slow as its slowest)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
+    """Rank r's independent copy of the workload (its own seed; heads never exchange data)."""
+    return w.with_(seed=w.seed + rank)
+
+
+def job_throughput(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens*heads/s: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 def barrier(world: int):
@@ -223,7 +234,7 @@ def run_blin(args, w):
     import block_causal_linear_rope_b200 as blin
 
     dt_t = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    wr = w.with_(seed=w.seed + rank)
+    wr = replica_workload(w, rank)
     q, k, v = workloads.call_tensors(wr)
     qh, kh, vh = (torch.from_numpy(x).to(dt_t).pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.to("cuda") for x in (qh, kh, vh))
@@ -301,8 +312,8 @@ def run_blin(args, w):
     e_ms = max_over_ranks(e_start.elapsed_time(e_end) / e_steps, world)
 
     units = w.B * w.H * w.N  # token*heads per GPU per step
-    value = units * world / (ms * 1e-3)
-    e2e_value = units * world / (e_ms * 1e-3)
+    value = job_throughput(units, world, ms)
+    e2e_value = job_throughput(units, world, e_ms)
 
     # ---- roofline of the dominant kernel (algorithmic bytes / live event time)
     elem = 2 if w.dtype == "bf16" else 4

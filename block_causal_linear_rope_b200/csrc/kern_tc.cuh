@@ -242,6 +242,9 @@ struct P1 {
     static constexpr int CTRL = 1024;
     static constexpr int FIXED = NL * 2 * TB + NO * 3 * TB + TB + CTRL + 1024;  // + RoPE table
     static constexpr int THREADS = 448;  // warps 0-7 transform, 8-11 epilogue, 12 producer, 13 MMA
+    // control block: mbarriers in the first 256 bytes, then the slot records
+    static_assert((2 * NL + 2 * NO + 3 * NACC) * 8 <= 256, "mbarriers overflow their 256-byte area");
+    static_assert(256 + 4 * (4 * NL + 4 * NO + NACC + 4) + 4 <= CTRL, "control block overflow");
 };
 
 // Persistent, one CTA per SM: CTA j takes chunks j, j + grid, ... (chunk-index
@@ -505,6 +508,9 @@ __global__ void __launch_bounds__(448, 1)
             const int u = flags[1];
             ptx::named_bar_sync(2, 128);  // everyone has read flags[1] before it is rewritten
             if (u < 0) break;
+            // each thread observes the accumulator's completion itself before
+            // reading TMEM (the phase is complete, so this returns at once)
+            if (!ptx::mbar_wait_bounded(accf(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) flags[0] = 1;
             ptx::tc_fence_after_sync();
             int bh, b, c;
             decode(u, bh, b, c);
@@ -870,7 +876,11 @@ __global__ void __launch_bounds__(608, 1)
             }
             ptx::named_bar_sync(bar_id, 128);
             const int valid = gf[0], trow0 = gf[1];
+            ptx::named_bar_sync(bar_id, 128);  // everyone has read gf before the leader rewrites it
             if (valid < 0) break;
+            // each thread observes the accumulator's completion itself before
+            // reading TMEM (the phase is complete, so this returns at once)
+            if (!ptx::mbar_wait_bounded(accf(e), n & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) flags[0] = 1;
             ptx::tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + e * C::ACOLS;
             float zh, zl;
