@@ -69,6 +69,10 @@ def _load() -> ctypes.CDLL:
     L.blin_version.restype = ctypes.c_char_p
     L.blin_set_timing_events.argtypes = [P, I]
     L.blin_set_timing_events.restype = I
+    L.blin_prefill_static.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), P, P]
+    L.blin_prefill_static.restype = I
+    L.blin_prefill_static_capacity.argtypes = []
+    L.blin_prefill_static_capacity.restype = S
     for fn in ("blin_state_init", "blin_state_free", "blin_state_reset", "blin_state_tensors",
                "blin_state_copy_to_host", "blin_state_copy_from_host", "blin_state_reserve",
                "blin_prefill", "blin_block_step", "blin_device_status"):

@@ -38,6 +38,8 @@ static blin_status fail(blin_status st, const char *fmt, ...) {
     return st;
 }
 
+blin_status blin::set_last_error(blin_status st, const char *msg) { return fail(st, "%s", msg); }
+
 static blin_status cuda_fail(cudaError_t e, const char *what) {
     return fail(BLIN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/blin.h"
+
 namespace blin {
 
 // Tokens per TMA tile / MMA row block, tiles per state chunk and per output CTA.
@@ -83,5 +85,8 @@ cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const
 
 // Device watchdog access.
 cudaError_t read_and_clear_watchdog(int *code);
+
+// Records `msg` as this thread's blin_last_error() text and returns `st`.
+blin_status set_last_error(blin_status st, const char *msg);
 
 }  // namespace blin

@@ -164,6 +164,34 @@ BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v
                             const int rope_split[3], float theta, float eps,
                             blin_state *st, int commit, blin_stream stream);
 
+/* ---------------------------------------------------------------- no allocation */
+
+/* blin_prefill for callers that cannot allocate device memory (the method on
+ * the SANA-Video pages has no counterpart; this is a library convenience).
+ * Some callers have no device allocator of their own -- for example a plugin
+ * inside a host framework that owns all device memory and hands out no
+ * scratch buffers -- so they cannot pass the workspace blin_prefill needs.
+ * This entry point takes the same arguments minus the workspace and uses a
+ * fixed scratch area of blin_prefill_static_capacity() bytes (32 MiB) that is
+ * part of the library's own device memory: every GPU that loads the library
+ * holds it until the process exits, and nothing is allocated per call.
+ *   - Shapes whose blin_prefill_workspace_size exceeds the capacity are
+ *     rejected with BLIN_ERR_WORKSPACE and a message naming both sizes.
+ *   - The first call on each device looks up the scratch area's device
+ *     address (cudaGetSymbolAddress with that device current); make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the one scratch area and it keeps the last
+ *     call's contents.  Nothing in it needs to start at zero (each call writes
+ *     everything it reads), but calls that overlap on the GPU, e.g. on two
+ *     streams at once, race on it: serialise them.
+ *   - Results are those of blin_prefill on the same arguments. */
+BLIN_API blin_status blin_prefill_static(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
+                                         int B, int H, int d, const blin_geom *g, blin_state *st,
+                                         blin_stream stream);
+
+/* Bytes of blin_prefill_static's fixed scratch area. */
+BLIN_API size_t blin_prefill_static_capacity(void);
+
 /* ---------------------------------------------------------------- status */
 
 /* Thread-local message for the last non-OK status of this thread ("" if none). */
