@@ -73,6 +73,8 @@ def _load() -> ctypes.CDLL:
     L.blin_prefill_static.restype = I
     L.blin_prefill_static_capacity.argtypes = []
     L.blin_prefill_static_capacity.restype = S
+    L.blin_launch_count.argtypes = []
+    L.blin_launch_count.restype = ctypes.c_ulonglong
     for fn in ("blin_state_init", "blin_state_free", "blin_state_reset", "blin_state_tensors",
                "blin_state_copy_to_host", "blin_state_copy_from_host", "blin_state_reserve",
                "blin_prefill", "blin_block_step", "blin_device_status"):
@@ -292,3 +294,8 @@ def device_status() -> int:
     if rc not in (0, -8):
         _check(rc)
     return code.value
+
+
+def launch_count() -> int:
+    """Kernels this library has launched in this process so far."""
+    return int(lib.blin_launch_count())

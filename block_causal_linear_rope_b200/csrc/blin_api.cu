@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/blin.h"
@@ -177,6 +178,9 @@ static bool make_map(CUtensorMap *m, const void *base, long long rows, int d) {
 // ---------------------------------------------------------------- launch sequence
 static thread_local cudaEvent_t const *g_timing = nullptr;
 
+// Kernels this library has launched in this process (all threads, all devices).
+static std::atomic<unsigned long long> g_launches{0};
+
 static void mark(int i, bool after, cudaStream_t s) {
     if (g_timing != nullptr) cudaEventRecord(g_timing[2 * i + (after ? 1 : 0)], s);
 }
@@ -203,18 +207,24 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
     cudaError_t e;
     mark(0, false, s);
     // the tensor-core kernels build their RoPE tables in shared memory themselves
-    if (!tc && (e = launch_rope_table(g, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
+    if (!tc) {
+        if ((e = launch_rope_table(g, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
     mark(0, true, s);
     mark(1, false, s);
     e = tc ? launch_partial_tc(g, d, mk, mv, s) : launch_partial_simt(g, d, bf, k, v, s);
     if (e != cudaSuccess) return cuda_fail(e, "partial-state launch");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(1, true, s);
     mark(2, false, s);
     if ((e = launch_scan(g, d, S_in, z_in, S_out, z_out, s)) != cudaSuccess) return cuda_fail(e, "scan launch");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(2, true, s);
     mark(3, false, s);
     e = tc ? launch_output_tc(g, d, mq, mo, o, s) : launch_output_simt(g, d, bf, q, o, s);
     if (e != cudaSuccess) return cuda_fail(e, "output launch");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(3, true, s);
     return BLIN_OK;
 }
@@ -436,6 +446,8 @@ blin_status blin_set_timing_events(void *const *events, int n) {
     g_timing = reinterpret_cast<cudaEvent_t const *>(events);
     return BLIN_OK;
 }
+
+unsigned long long blin_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 blin_status blin_device_status(int *code) {
     int c = 0;

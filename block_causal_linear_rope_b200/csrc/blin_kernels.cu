@@ -106,6 +106,9 @@ static cudaError_t set_smem(int bytes) {
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    // the largest shared-memory carveout, so that two CTAs of ~113 KB fit on an SM
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 227 * 1024;
     return e;
 }
@@ -181,9 +184,12 @@ cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, cons
     if (wd == nullptr) return cudaErrorInvalidDevice;
     const long long units = (long long)g.cpb * g.nblk * g.BH;
     const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
+    // a CTA runs NP pipelines, each taking every NP-th of the CTA's chunks
     if (d == 32)
-        return launch_persistent<partial_tc_kernel<32, 4, 6, 6>>(false, P1<32>::FIXED + tab, P1<32>::THREADS, units, s, mk, mv, g, wd);
-    return launch_persistent<partial_tc_kernel<64, 8, 12, 12>>(false, P1<64>::FIXED + tab, P1<64>::THREADS, units, s, mk, mv, g, wd);
+        return launch_persistent<partial_tc_kernel<32, 4, 6, 6>>(false, P1<32>::FIXED + tab, P1<32>::THREADS,
+                                                                 (units + P1<32>::NP - 1) / P1<32>::NP, s, mk, mv, g, wd);
+    return launch_persistent<partial_tc_kernel<64, 8, 12, 12>>(false, P1<64>::FIXED + tab, P1<64>::THREADS,
+                                                               (units + P1<64>::NP - 1) / P1<64>::NP, s, mk, mv, g, wd);
 }
 
 cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo,

@@ -76,24 +76,42 @@ struct TokPos {
     }
 };
 
-// Where a CTA reads RoPE (cos, sin) pairs from: its shared-memory copy (frame
-// window + full y and x tables) when the call's tables are small, else the
-// global table.
+// A CTA's shared-memory RoPE table: (cos, sin) of every (position, pair) of
+// the call's frame window and of every row and column, one section per axis.
+// Each section is stored pair-major ([pair][position]) so that the threads of
+// a warp, which hold consecutive tokens and hence mostly consecutive columns,
+// read consecutive words: no bank conflicts on the x section, broadcasts on t, y.
 struct RopeTab {
     const float2 *t, *y, *x;  // t indexed by relative frame (window offset folded in)
+    int nt, ny, nx;            // positions per pair in each section (T, Hg, Wg)
 };
 
-// Fills this CTA's shared-memory copy of the call's RoPE table (the
-// tensor-core path is only chosen when it fits; transform threads only, a
-// barrier among them must follow).
+// Fills this CTA's shared-memory RoPE table (the tensor-core path is only
+// chosen when it fits; transform threads only, a barrier among them must
+// follow).  Entry values are those of rope_entry (same order of operations).
 template <int PT, int PY, int PX>
 __device__ __forceinline__ RopeTab load_rope_tab(const KGeom &g, float2 *s_tab, int tid, int nthreads) {
-    const int n = g.T * PT + g.Hg * PY + g.Wg * PX;
-    for (int i = tid; i < n; i += nthreads) s_tab[i] = rope_entry(i, g.T, g.t0, g.Hg, PT, PY, PX, g.theta);
+    const int nt = g.T * PT, ny = g.Hg * PY, n = nt + ny + g.Wg * PX;
+    for (int i = tid; i < n; i += nthreads) {
+        int src;  // index of the same entry in the position-major order rope_entry enumerates
+        if (i < nt) {
+            src = (i % g.T) * PT + i / g.T;
+        } else if (i < nt + ny) {
+            const int r = i - nt;
+            src = nt + (r % g.Hg) * PY + r / g.Hg;
+        } else {
+            const int r = i - nt - ny;
+            src = nt + ny + (r % g.Wg) * PX + r / g.Wg;
+        }
+        s_tab[i] = rope_entry(src, g.T, g.t0, g.Hg, PT, PY, PX, g.theta);
+    }
     RopeTab r;
     r.t = s_tab;
     r.y = s_tab + g.tab_y;
     r.x = s_tab + g.tab_x;
+    r.nt = g.T;
+    r.ny = g.Hg;
+    r.nx = g.Wg;
     return r;
 }
 
@@ -106,12 +124,12 @@ template <int D, int PT, int PY, int PX, bool ZP>
 __device__ __forceinline__ void phi_rope_row(uint32_t (&w)[D / 2], uint32_t (&ph)[D / 2], const RopeTab &tab,
                                              const TokPos &tp, float *zp) {
     static_assert(PT + PY + PX == D / 2, "split must cover d");
-    const float2 *rt = tab.t + tp.t * PT;
-    const float2 *ry = tab.y + tp.y * PY;
-    const float2 *rx = tab.x + tp.x * PX;
+    const float2 *rt = tab.t + tp.t;
+    const float2 *ry = tab.y + tp.y;
+    const float2 *rx = tab.x + tp.x;
 #pragma unroll
     for (int p = 0; p < D / 2; ++p) {
-        const float2 cs = p < PT ? rt[p] : (p < PT + PY ? ry[p - PT] : rx[p - PT - PY]);
+        const float2 cs = p < PT ? rt[p * tab.nt] : (p < PT + PY ? ry[(p - PT) * tab.ny] : rx[(p - PT - PY) * tab.nx]);
         // ReLU on the packed pair (exact), then widen
         __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162 *>(&w[p]);
         hv = __hmax2(hv, __float2bfloat162_rn(0.f));
@@ -226,6 +244,13 @@ __device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_c
 // other group, which just stops.
 constexpr int kEndFirst = -1, kEndSecond = -2;
 
+// One mbarrier arrival for the whole warp, after every lane's shared-memory
+// accesses (and tcgen05 loads, fenced by the caller) are ordered before it.
+__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar);
+}
+
 // ============================================================================ pass 1
 template <int D>
 struct P1 {
@@ -233,60 +258,76 @@ struct P1 {
     static constexpr int TB = kTile * ROWB;
     static constexpr int M = D == 32 ? 64 : 128;          // [K~^T ; phi(K)^T]
     static constexpr int N = D == 32 ? D + 8 : D + 16;   // [V | ones]
-    static constexpr int NL = D == 32 ? 7 : 2;           // landing stages: K | V (TMA)
-    static constexpr int NO = D == 32 ? 3 : 2;           // operand sets: K~ | phi | V
-    static constexpr int NACC = 4;                       // TMEM accumulators (chunks in flight)
+    static constexpr int NP = D == 32 ? 2 : 1;           // independent pipelines per CTA (MMA issuers)
+    static constexpr int NL = D == 32 ? 4 : 3;           // landing stages per pipeline: K | V; V is read by the MMA
+    static constexpr int NO = 2;                         // operand sets per pipeline: K~ | phi
+    static constexpr int NACC = 2;                       // TMEM accumulators per pipeline (chunks in flight)
     static constexpr int ACOLS = D == 32 ? 64 : 128;     // TMEM columns per accumulator
-    static constexpr uint32_t TCOLS = NACC * ACOLS;
+    static constexpr uint32_t TCOLS = NP * NACC * ACOLS;
     static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
+    static constexpr int NBAR = 2 * NL + 2 * NO + 2 * NACC;  // mbarriers per pipeline
     static constexpr int CTRL = 1024;
-    static constexpr int FIXED = NL * 2 * TB + NO * 3 * TB + TB + CTRL + 1024;  // + RoPE table
-    static constexpr int THREADS = 448;  // warps 0-7 transform, 8-11 epilogue, 12 producer, 13 MMA
-    // control block: mbarriers in the first 256 bytes, then the slot records
-    static_assert((2 * NL + 2 * NO + 3 * NACC) * 8 <= 256, "mbarriers overflow their 256-byte area");
-    static_assert(256 + 4 * (4 * NL + 4 * NO + NACC + 4) + 4 <= CTRL, "control block overflow");
+    static constexpr int BARS = 512;                     // mbarrier area at the start of the control block
+    static constexpr int FIXED = NP * (NL + NO) * 2 * TB + TB + CTRL + 1024;  // + RoPE table
+    static constexpr int THREADS = 32 * 6 * NP;  // warps [0, 4NP) transform, then NP producers, NP MMA issuers
+    static_assert(NP * NBAR * 8 <= BARS, "mbarriers overflow their area");
+    static_assert(BARS + 4 * NP * (4 * NL + 4 * NO) + 16 <= CTRL, "control block overflow");
+    // the B operand's second N atom (the ones block) sits above every landing slot
+    static_assert(NP * (NL + NO) * 2 * TB - TB < (1 << 18), "LBO field range");
+    static_assert(TCOLS <= 512, "TMEM holds 512 columns");
 };
 
-// Persistent, one CTA per SM: CTA j takes chunks j, j + grid, ... (chunk-index
-// major, so the short last chunk of every block comes last and spreads evenly).  TMA lands K and V tiles in a deep ring; transform warps
-// release each landing slot as soon as they have read it and write the MMA
-// operands (K~, phi(K), V) into a second ring, so DRAM latency is covered by
-// the landing ring alone.  Four TMEM accumulators let chunk epilogues
-// (TMEM -> chunk partial in global memory) trail the MMAs.
+// Persistent, one CTA per SM (a kernel that uses tcgen05 gets one CTA per SM).
+// The CTA runs NP independent pipelines, so that NP threads issue MMAs: one
+// thread issues a tcgen05.mma about every 50 cycles and the eight M = 64 MMAs
+// a 128-token tile needs from one thread would not keep up with HBM, while two
+// issuers' MMAs overlap in the tensor core.  Pipeline p takes every other
+// chunk of the CTA's static round robin (chunks j, j + grid, ..., chunk-index
+// major so the short last chunk of every block comes last and spreads evenly).
+// Per pipeline: a producer thread lands K and V tiles with TMA; four
+// transform warps read K and write the A operand (K~, phi(K)) into an operand
+// ring; an MMA thread accumulates [K~^T; phi^T] x [V | 1] into a TMEM
+// accumulator per chunk, taking V straight from the landing slot (a slot is
+// free after 5 arrivals: 4 transform warps + 1 commit).  Two tiles into the
+// next chunk, the transform warps read the finished accumulator back (each warp
+// its TMEM subpartition) and write the chunk partial to global memory.
 template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(P1<D>::THREADS, 1)
     partial_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                       KGeom g, int *watchdog) {
     using C = P1<D>;
-    constexpr int NL = C::NL, NO = C::NO, TB = C::TB, ROWB = C::ROWB, E = D * D + D;
+    constexpr int NP = C::NP, NL = C::NL, NO = C::NO, NA = C::NACC, TB = C::TB, ROWB = C::ROWB, E = D * D + D;
     constexpr uint32_t IDESC = ptx::idesc_bf16_f32(C::M, C::N, 1, 1);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *land = smem;                       // [NL][K | V]
-    uint8_t *opnd = land + NL * 2 * TB;         // [NO][K~ | phi | V]
-    uint8_t *ones = opnd + NO * 3 * TB;         // constant B block
+    uint8_t *land0 = smem;                         // [NP][NL][K | V]
+    uint8_t *opnd0 = land0 + NP * NL * 2 * TB;     // [NP][NO][K~ | phi]
+    uint8_t *ones = opnd0 + NP * NO * 2 * TB;      // constant B block (above every V tile: positive LBO)
     uint8_t *ctrl = ones + TB;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
-    int *linfo = reinterpret_cast<int *>(ctrl + 256);                 // [NL][4] unit, tile, valid, last
-    int *oinfo = linfo + 4 * NL;                                      // [NO][4]
-    int *acc_unit = oinfo + 4 * NO;                                   // [NACC]
-    volatile int *flags = reinterpret_cast<volatile int *>(acc_unit + C::NACC);  // abort, epilogue
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_unit + C::NACC + 4);
+    volatile int *flags = reinterpret_cast<volatile int *>(ctrl + C::BARS);  // [0] abort
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + C::BARS + 4);
+    int *info0 = reinterpret_cast<int *>(ctrl + C::BARS + 16);          // [NP][NL + NO][4]
     float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // this thread's pipeline
+    const int pipe = warp < 4 * NP ? warp >> 2 : (warp - 4 * NP) % NP;
+    uint8_t *land = land0 + pipe * NL * 2 * TB;
+    uint8_t *opnd = opnd0 + pipe * NO * 2 * TB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl) + pipe * C::NBAR;
+    int *linfo = info0 + pipe * 4 * (NL + NO);  // [NL][4] unit, tile, valid, last
+    int *oinfo = linfo + 4 * NL;                 // [NO][4]
     auto lk = [&](int s) { return land + s * 2 * TB; };
     auto lv = [&](int s) { return land + s * 2 * TB + TB; };
-    auto ok_ = [&](int s) { return opnd + s * 3 * TB; };
-    auto op_ = [&](int s) { return opnd + s * 3 * TB + TB; };
-    auto ov_ = [&](int s) { return opnd + s * 3 * TB + 2 * TB; };
+    auto ok_ = [&](int s) { return opnd + s * 2 * TB; };
+    auto op_ = [&](int s) { return opnd + s * 2 * TB + TB; };
     auto lfull = [&](int s) { return ptx::smem_u32(bars + s); };
     auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
     auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
     auto oempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
-    constexpr int NA = C::NACC;
     auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + a); };
-    auto accp = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + NA + a); };
-    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 2 * NA + a); };
+    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + NA + a); };
 
     const int units = g.cpb * g.nblk * g.BH;
     const int per_c = g.nblk * g.BH;
@@ -298,20 +339,21 @@ __global__ void __launch_bounds__(448, 1)
         b = rem - bh * g.nblk;
     };
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < NL; ++s) {
-            ptx::mbar_init(lfull(s), 1);
-            ptx::mbar_init(lempty(s), 128);
-        }
-        for (int s = 0; s < NO; ++s) {
-            ptx::mbar_init(ofull(s), 128);
-            ptx::mbar_init(oempty(s), 1);
-        }
-        for (int a = 0; a < NA; ++a) {
-            ptx::mbar_init(accf(a), 1);
-            ptx::mbar_init(accp(a), 1);
-            ptx::mbar_init(acce(a), 128);
+        for (int p = 0; p < NP; ++p) {
+            uint64_t *pb = reinterpret_cast<uint64_t *>(ctrl) + p * C::NBAR;
+            for (int s = 0; s < NL; ++s) {
+                ptx::mbar_init(ptx::smem_u32(pb + s), 1);
+                ptx::mbar_init(ptx::smem_u32(pb + NL + s), 5);  // 4 transform warps (K read) + MMA commit (V read)
+            }
+            for (int s = 0; s < NO; ++s) {
+                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + s), 4);  // one arrival per transform warp
+                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + NO + s), 1);
+            }
+            for (int a = 0; a < NA; ++a) {
+                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + 2 * NO + a), 1);
+                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + 2 * NO + NA + a), 4);  // one arrival per transform warp
+            }
         }
         flags[0] = 0;
         ptx::fence_mbar_init();
@@ -323,17 +365,17 @@ __global__ void __launch_bounds__(448, 1)
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot + pipe * NA * C::ACOLS;  // this pipeline's accumulators
     if (tid == 0) griddep_launch_dependents();
 
-    if (warp == 12) {
+    if (warp >= 4 * NP && warp < 5 * NP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ptx::tma_prefetch_map(&mk);
             ptx::tma_prefetch_map(&mv);
             int k = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {  // static round robin
+            for (int u = blockIdx.x + pipe * gridDim.x; ok && u < units; u += NP * gridDim.x) {  // static round robin
                 int bh, b, c;
                 decode(u, bh, b, c);
                 const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
@@ -359,25 +401,23 @@ __global__ void __launch_bounds__(448, 1)
                     }
                 }
             }
-            for (int e = 0; ok && e < 2; ++e, ++k) {  // end markers, one per transform group
-                const int sl = k % NL;
-                if (k >= NL && !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
-                                                       kWaitLimitNs))
-                    break;
-                linfo[4 * sl] = e == 0 ? kEndFirst : kEndSecond;
+            // end marker for the transform warps
+            const int sl = k % NL;
+            if (ok && (k < NL || ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
+                                                        kWaitLimitNs))) {
+                linfo[4 * sl] = kEndFirst;
                 ptx::mbar_arrive(lfull(sl));
             }
         }
-    } else if (warp == 13) {
+    } else if (warp >= 5 * NP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int nu = 0;
-            bool ok = true;
             for (int k = 0;; ++k) {
                 const int so = k % NO;
                 if (flags[0] ||
                     !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
-                    ok = false;
+                    flags[0] = 1;
                     break;
                 }
                 const int *inf = oinfo + 4 * so;
@@ -386,132 +426,49 @@ __global__ void __launch_bounds__(448, 1)
                 const int a = nu % NA;
                 if (t == 0 && nu >= NA &&
                     !ptx::mbar_wait_bounded(acce(a), ((nu / NA) - 1) & 1, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
-                    ok = false;
+                    flags[0] = 1;
                     break;
                 }
                 ptx::tc_fence_after_sync();
-                const uint32_t ka = ptx::smem_u32(ok_(so)), va = ptx::smem_u32(ov_(so));
-                const uint32_t lbo_b = ptx::smem_u32(ones) - va;  // N atom 1 = the ones block
+                const int sl = k % NL;  // the tile's landing slot (same tile order as the producer)
+                const uint32_t va = ptx::smem_u32(lv(sl));
+                // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones.
+                // Consecutive K steps are 16 token rows (16 * ROWB bytes: ROWB in the address field).
+                const uint64_t ad = ptx::smem_desc(ptx::smem_u32(ok_(so)), TB, 8 * ROWB, C::LAYOUT);
+                const uint64_t bd = ptx::smem_desc(va, ptx::smem_u32(ones) - va, 8 * ROWB, C::LAYOUT);
+                const uint32_t dacc = tmem + a * C::ACOLS;
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones
-                    const uint64_t ad = ptx::smem_desc(ka + kk * 16 * ROWB, TB, 8 * ROWB, C::LAYOUT);
-                    const uint64_t bd = ptx::smem_desc(va + kk * 16 * ROWB, lbo_b, 8 * ROWB, C::LAYOUT);
-                    ptx::mma_bf16_ss(tmem + a * C::ACOLS, ad, bd, IDESC, (t > 0 || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    ptx::mma_bf16_ss(dacc, ad + static_cast<uint64_t>(kk * ROWB), bd + static_cast<uint64_t>(kk * ROWB),
+                                     IDESC, (t > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(oempty(so));
+                ptx::mma_commit(lempty(sl));
                 if (last) {
-                    acc_unit[a] = u;
-                    ptx::mbar_arrive(accp(a));
                     ptx::mma_commit(accf(a));
                     ++nu;
                 }
             }
-            if (!ok) flags[0] = 1;
-            const int a = nu % NA;  // tell the epilogue there is nothing more
-            if (ok && (nu < NA || ptx::mbar_wait_bounded(acce(a), ((nu / NA) - 1) & 1, watchdog, WD_PARTIAL_ACC,
-                                                         kWaitLimitNs))) {
-                acc_unit[a] = -1;
-                ptx::mbar_arrive(accp(a));
-            }
         }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ transform warps (two groups)
-        const int grp = warp >> 2, r = tid & 127;
-        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 256);
+    } else {
+        // ------------------------------------------------------------ transform warps: one row per thread
+        const int r = tid & 127, sub = warp & 3;
+        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 128 * NP);
         {
             uint4 *o4 = reinterpret_cast<uint4 *>(ones);  // all 1.0, so its swizzle is irrelevant
-            for (int i = tid; i < TB / 16; i += 256) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+            for (int i = tid; i < TB / 16; i += 128 * NP) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
         }
-        ptx::named_bar_sync(1, 256);
-        const int step = 2 * kTile;
-        const int dx = step % g.Wg, dy = (step / g.Wg) % g.Hg, dt = step / g.HW;
-        TokPos tp{0, 0, 0};
-        for (int k = grp;; k += 2) {
-            const int sl = k % NL, so = k % NO;
-            if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs)) {
-                flags[0] = 1;
-                break;
-            }
-            const int *inf = linfo + 4 * sl;
-            const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
-            const int last = ld_volatile(inf + 3);
-            if (u == kEndSecond) break;
-            // read this row of the landed tiles and give the slot back right away
-            uint32_t w[D / 2], vw[D / 2], ph[D / 2];
-            const bool live = u >= 0 && r < valid;
-            if (live) {
-                load_row<D>(lk(sl), r, w);
-                load_row<D>(lv(sl), r, vw);
-            }
-            if (u >= 0) ptx::mbar_arrive(lempty(sl));
-            if (k >= NO &&
-                !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
-                flags[0] = 1;
-                break;
-            }
-            if (u == kEndFirst) {  // pass the end on to the MMA issuer, in operand order
-                if (r == 0) oinfo[4 * so] = kEndFirst;
-                ptx::mbar_arrive(ofull(so));
-                break;
-            }
-            if (t <= 1) {
-                int bh, b, c;
-                decode(u, bh, b, c);
-                tp.init(g, block_frame_begin(g, b) * g.HW + c * kChunk + t * kTile + r);
-            } else {
-                tp.advance(g, dx, dy, dt);
-            }
-            if (live) {
-                phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
-                store_row<D>(ok_(so), r, w);
-                store_row<D>(op_(so), r, ph);
-                store_row<D>(ov_(so), r, vw);
-            } else {  // rows past the chunk add nothing
-                zero_row<D>(ok_(so), r);
-                zero_row<D>(op_(so), r);
-                zero_row<D>(ov_(so), r);
-            }
-            ptx::fence_proxy_async_smem();
-            if (r == 0) {
-                int *oi = oinfo + 4 * so;
-                oi[0] = u;
-                oi[1] = t;
-                oi[2] = valid;
-                oi[3] = last;
-            }
-            ptx::mbar_arrive(ofull(so));
-        }
-    } else if (warp < 12) {
-        // ------------------------------------------------------------ epilogue warps (8-11)
-        const int er = tid - 256, sub = warp & 3;
-        // M = 64 (d = 32): accumulator row m in TMEM lane (m % 16) + 32 * (m / 16);
-        // M = 128 (d = 64): row m in lane m.  Rows [0, D) hold P, rows [D, 2D) hold
-        // phi^T against the ones block, i.e. zp, in column D.
-        constexpr int RPS = D == 32 ? 16 : 32;  // accumulator rows per TMEM subpartition
-        for (int nu = 0;; ++nu) {
-            const int a = nu % NA, ph = (nu / NA) & 1;
-            if (er == 0) {  // one thread waits and decides for all 128 (named barrier below)
-                int u = -1;
-                if (!flags[0] && ptx::mbar_wait_bounded(accp(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
-                    u = ld_volatile(acc_unit + a);
-                    if (u >= 0 && !ptx::mbar_wait_bounded(accf(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
-                        u = -1;
-                        flags[0] = 1;
-                    }
-                } else {
-                    flags[0] = 1;
-                }
-                flags[1] = u;
-            }
-            ptx::named_bar_sync(2, 128);
-            const int u = flags[1];
-            ptx::named_bar_sync(2, 128);  // everyone has read flags[1] before it is rewritten
-            if (u < 0) break;
-            // each thread observes the accumulator's completion itself before
-            // reading TMEM (the phase is complete, so this returns at once)
+        ptx::fence_proxy_async_smem();  // the ones block is read by the MMA (async proxy)
+        ptx::named_bar_sync(1, 128 * NP);
+
+        // Chunk epilogue (each warp its TMEM subpartition): accumulator -> chunk
+        // partial.  M = 64 (d = 32): accumulator row m in TMEM lane
+        // (m % 16) + 32 * (m / 16); M = 128 (d = 64): row m in lane m.  Rows
+        // [0, D) hold P, rows [D, 2D) hold phi^T against the ones block, i.e. zp,
+        // in column D.
+        auto epilogue = [&](int u, int a, int ph) {
             if (!ptx::mbar_wait_bounded(accf(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) flags[0] = 1;
             ptx::tc_fence_after_sync();
+            constexpr int RPS = D == 32 ? 16 : 32;  // accumulator rows per TMEM subpartition
             int bh, b, c;
             decode(u, bh, b, c);
             float *out = g.part + ((size_t)(bh * g.nblk + b) * g.cpb + c) * E;
@@ -534,14 +491,87 @@ __global__ void __launch_bounds__(448, 1)
                 if (lane < RPS) out[D * D + RPS * (sub - 2) + lane] = zv;
             }
             ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(acce(a));  // accumulator a is free again
+            warp_arrive(acce(a), lane);  // accumulator a is free again
+        };
+
+        const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
+        TokPos tp{0, 0, 0};
+        int nu = 0;                               // chunks pushed to the MMA so far
+        int pend_u = -1, pend_a = 0, pend_ph = 0;  // finished chunk whose epilogue is still due
+        int since = 0;                            // tiles pushed since that chunk's last tile
+        for (int k = 0;; ++k) {
+            const int sl = k % NL, so = k % NO;
+            if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            const int *inf = linfo + 4 * sl;
+            const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
+            const int last = ld_volatile(inf + 3);
+            // read this row of K; rows past the chunk also clear their V row
+            // (the MMA reads V in place: other blocks' tokens must add nothing)
+            uint32_t w[D / 2], ph[D / 2];
+            const bool live = u >= 0 && r < valid;
+            if (live) load_row<D>(lk(sl), r, w);
+            else if (u >= 0) zero_row<D>(lv(sl), r);
+            if (u >= 0) {
+                if (valid < kTile) ptx::fence_proxy_async_smem();
+                warp_arrive(lempty(sl), lane);
+            }
+            if (k >= NO &&
+                !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
+                flags[0] = 1;
+                break;
+            }
+            if (u < 0) {  // pass the end on to the MMA issuer, in operand order
+                if (r == 0) oinfo[4 * so] = kEndFirst;
+                warp_arrive(ofull(so), lane);
+                break;
+            }
+            if (t == 0) {
+                int bh, b, c;
+                decode(u, bh, b, c);
+                tp.init(g, block_frame_begin(g, b) * g.HW + c * kChunk + r);
+            } else {
+                tp.advance(g, dx, dy, dt);
+            }
+            if (live) {
+                phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
+                store_row<D>(ok_(so), r, w);
+                store_row<D>(op_(so), r, ph);
+            } else {  // rows past the chunk add nothing
+                zero_row<D>(ok_(so), r);
+                zero_row<D>(op_(so), r);
+            }
+            ptx::fence_proxy_async_smem();
+            if (r == 0) {
+                int *oi = oinfo + 4 * so;
+                oi[0] = u;
+                oi[1] = t;
+                oi[2] = valid;
+                oi[3] = last;
+            }
+            warp_arrive(ofull(so), lane);
+            // the previous chunk's epilogue, once its MMAs have had two tiles' time
+            if (pend_u >= 0 && (++since >= 2 || last)) {
+                epilogue(pend_u, pend_a, pend_ph);
+                pend_u = -1;
+            }
+            if (last) {
+                pend_u = u;
+                pend_a = nu % NA;
+                pend_ph = (nu / NA) & 1;
+                since = 0;
+                ++nu;
+            }
         }
+        if (pend_u >= 0 && !flags[0]) epilogue(pend_u, pend_a, pend_ph);
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem, C::TCOLS);
+        ptx::tmem_dealloc(*tmem_slot, C::TCOLS);
     }
 }
 
@@ -557,23 +587,26 @@ struct P2 {
     static constexpr int BATOM = OutB<D>::BATOM;       // one K atom of B (N rows)
     static constexpr int IMG = OutB<D>::IMG;
     static constexpr int ACOLS = D == 32 ? 64 : 128;   // TMEM columns per accumulator
-    static constexpr uint32_t TCOLS = 2 * ACOLS;
+    static constexpr int NACC = 4;                     // TMEM accumulators; epilogue group e uses e, e + 2
+    static constexpr uint32_t TCOLS = NACC * ACOLS;
     static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
     static constexpr int PRE = (D * D + D) * 4;        // one fp32 prefix state (S, z)
-    static constexpr int NBARS = 2 * NL + 2 * NO + 12;
+    static constexpr int NBARS = 2 * NL + 2 * NO + 3 * NACC + 6;
     static constexpr int INFO = (NBARS * 8 + 15) / 16 * 16;
     static constexpr int CTRL = 1024;
     static constexpr int FIXED = NL * TB + NO * 2 * TB + 2 * NSTG * TB + 2 * IMG + 2 * PRE + CTRL + 1024;  // + table
     static constexpr int THREADS = 608;  // warps 0-7 transform, 8-15 epilogue, 16 producer, 17 MMA, 18 B prep
-    static_assert(INFO + 32 * NL + 32 * NO + 32 + 64 + 16 <= CTRL, "control block overflow");
+    static_assert(INFO + 32 * NL + 32 * NO + 16 * NACC + 64 + 16 <= CTRL, "control block overflow");
+    static_assert(TCOLS <= 512, "TMEM holds 512 columns");
 };
 
 // Persistent, one CTA per SM: CTA j takes groups j, j + grid, ... of <= 8 query
 // tiles of one (head, block).  Per group the
 // producer bulk-copies the fp32 prefix state, which a B-prep warp turns into
 // the bf16 B operand (both double-buffered); per tile it lands Q in a deep ring.  Two transform groups write [R phi(q) | phi(q)] into
-// an operand ring; the MMA issuer alternates two TMEM accumulators, and
-// epilogue group e (warps 8+4e..11+4e) owns accumulator e: it divides, writes
+// an operand ring; the MMA issuer cycles through four TMEM accumulators, and
+// epilogue group e (warps 8+4e..11+4e) takes tiles of parity e (accumulators e
+// and e + 2), so an MMA never waits on the epilogue of the tile just before it: it divides, writes
 // bf16 rows to its staging buffer and stores them with TMA (plain stores for a
 // ragged tile).
 template <int D, int PT, int PY, int PX>
@@ -595,9 +628,9 @@ __global__ void __launch_bounds__(608, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
     int *linfo = reinterpret_cast<int *>(ctrl + C::INFO);  // [NL][8]: unit, tile, valid, ord, row0, last
     int *oinfo = linfo + 8 * NL;                          // [NO][8]
-    int *ainfo = oinfo + 8 * NO;                          // [2][4]: valid (-1 = end), row0
-    volatile int *flags = reinterpret_cast<volatile int *>(ainfo + 8);  // [0] abort, [2..3] prefix slots, [4+4e..]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ainfo + 8 + 16);
+    int *ainfo = oinfo + 8 * NO;                          // [NACC][4]: valid (-1 = end), row0
+    volatile int *flags = reinterpret_cast<volatile int *>(ainfo + 4 * C::NACC);  // [0] abort, [2..3] prefix slots, [4+4e..]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ainfo + 4 * C::NACC + 16);
     float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
     auto lq = [&](int s) { return land + s * TB; };
     auto oq = [&](int s) { return opnd + s * 2 * TB; };
@@ -606,12 +639,13 @@ __global__ void __launch_bounds__(608, 1)
     auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
     auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
     auto oempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
-    auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + a); };
-    auto accp = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 2 + a); };
-    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 4 + a); };
-    auto bfull = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 6 + a); };
-    auto bempty = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 8 + a); };
-    auto pfull = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + 10 + a); };
+    constexpr int NA = C::NACC, AB = 2 * NL + 2 * NO;
+    auto accf = [&](int a) { return ptx::smem_u32(bars + AB + a); };
+    auto accp = [&](int a) { return ptx::smem_u32(bars + AB + NA + a); };
+    auto acce = [&](int a) { return ptx::smem_u32(bars + AB + 2 * NA + a); };
+    auto bfull = [&](int a) { return ptx::smem_u32(bars + AB + 3 * NA + a); };
+    auto bempty = [&](int a) { return ptx::smem_u32(bars + AB + 3 * NA + 2 + a); };
+    auto pfull = [&](int a) { return ptx::smem_u32(bars + AB + 3 * NA + 4 + a); };
 
     const int units = g.qcpb * g.nblk * g.BH;
     const int per_q = g.nblk * g.BH;
@@ -627,16 +661,18 @@ __global__ void __launch_bounds__(608, 1)
     if (tid == 0) {
         for (int s = 0; s < NL; ++s) {
             ptx::mbar_init(lfull(s), 1);
-            ptx::mbar_init(lempty(s), 128);
+            ptx::mbar_init(lempty(s), 4);  // one arrival per transform warp
         }
         for (int s = 0; s < NO; ++s) {
-            ptx::mbar_init(ofull(s), 128);
+            ptx::mbar_init(ofull(s), 4);
             ptx::mbar_init(oempty(s), 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < NA; ++a) {
             ptx::mbar_init(accf(a), 1);
             ptx::mbar_init(accp(a), 1);
-            ptx::mbar_init(acce(a), 128);
+            ptx::mbar_init(acce(a), 4);  // one arrival per epilogue warp
+        }
+        for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(bfull(a), 1);
             ptx::mbar_init(bempty(a), 1);
             ptx::mbar_init(pfull(a), 1);
@@ -745,7 +781,7 @@ __global__ void __launch_bounds__(608, 1)
             bool ok = true;
             int k = 0;
             for (;; ++k) {
-                const int so = k % NO, a = k & 1;
+                const int so = k % NO, a = k % NA;
                 if (flags[0] || !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
                     ok = false;
                     break;
@@ -754,8 +790,8 @@ __global__ void __launch_bounds__(608, 1)
                 const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
                 const int ord = ld_volatile(inf + 3), row0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
                 if (u < 0) break;
-                if ((k >= 2 &&
-                     !ptx::mbar_wait_bounded(acce(a), ((k >> 1) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs)) ||
+                if ((k >= NA &&
+                     !ptx::mbar_wait_bounded(acce(a), ((k / NA) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs)) ||
                     (t == 0 &&
                      !ptx::mbar_wait_bounded(bfull(ord & 1), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))) {
                     ok = false;
@@ -782,9 +818,9 @@ __global__ void __launch_bounds__(608, 1)
             if (!ok) flags[0] = 1;
             // tell both epilogue groups there is nothing more (tiles k and k + 1)
             for (int j = 0; ok && j < 2; ++j) {
-                const int kk = k + j, a = kk & 1;
-                if (kk >= 2 &&
-                    !ptx::mbar_wait_bounded(acce(a), ((kk >> 1) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs))
+                const int kk = k + j, a = kk % NA;
+                if (kk >= NA &&
+                    !ptx::mbar_wait_bounded(acce(a), ((kk / NA) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs))
                     break;
                 ainfo[4 * a] = -1;
                 ptx::mbar_arrive(accp(a));
@@ -812,7 +848,7 @@ __global__ void __launch_bounds__(608, 1)
             uint32_t w[D / 2], ph[D / 2];
             const bool live = u >= 0 && r < valid;
             if (live) load_row<D>(lq(sl), r, w);
-            if (u >= 0) ptx::mbar_arrive(lempty(sl));  // landing slot read
+            if (u >= 0) warp_arrive(lempty(sl), lane);  // landing slot read
             if (k >= NO &&
                 !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
                 flags[0] = 1;
@@ -820,7 +856,7 @@ __global__ void __launch_bounds__(608, 1)
             }
             if (u == kEndFirst) {  // pass the end on to the MMA issuer, in operand order
                 if (r == 0) oinfo[8 * so] = kEndFirst;
-                ptx::mbar_arrive(ofull(so));
+                warp_arrive(ofull(so), lane);
                 break;
             }
             if (t <= 1) {
@@ -848,7 +884,7 @@ __global__ void __launch_bounds__(608, 1)
                 oi[4] = row0;
                 oi[5] = last;
             }
-            ptx::mbar_arrive(ofull(so));
+            warp_arrive(ofull(so), lane);
         }
     } else {
         // ------------------------------------------------------------ epilogue groups (warps 8-15)
@@ -856,33 +892,35 @@ __global__ void __launch_bounds__(608, 1)
         const int r = 32 * sub + lane;  // tile row read back by this thread (TMEM subpartition)
         volatile int *gf = flags + 4 + 4 * e;
         const uint32_t bar_id = 2 + e;
-        for (int n = 0;; ++n) {  // this group's n-th tile uses accumulator e
+        for (int n = 0;; ++n) {  // this group's n-th tile is tile k = 2n + e, in accumulator k % NACC
+            const int a = (2 * n + e) % NA, aph = ((2 * n + e) / NA) & 1;
             if (er == 0) {  // one thread waits and decides for the group (named barrier below)
                 int valid = -1;
-                if (!flags[0] && ptx::mbar_wait_bounded(accp(e), n & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
-                    valid = ld_volatile(ainfo + 4 * e);
-                    gf[1] = ld_volatile(ainfo + 4 * e + 1);
+                if (!flags[0] && ptx::mbar_wait_bounded(accp(a), aph, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
+                    valid = ld_volatile(ainfo + 4 * a);
+                    gf[2 * (n & 1) + 1] = ld_volatile(ainfo + 4 * a + 1);
                     if (valid >= 0 &&
-                        !ptx::mbar_wait_bounded(accf(e), n & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
+                        !ptx::mbar_wait_bounded(accf(a), aph, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
                         valid = -1;
                         flags[0] = 1;
                     }
                 } else {
                     flags[0] = 1;
                 }
-                gf[0] = valid;
+                gf[2 * (n & 1)] = valid;
                 // the staging buffer about to be reused has been read by its TMA store
                 ptx::bulk_wait_group_read<NSTG - 1>();
             }
+            // the record alternates between two slots, so one barrier suffices:
+            // the leader rewrites slot n & 1 only after barrier n + 1
             ptx::named_bar_sync(bar_id, 128);
-            const int valid = gf[0], trow0 = gf[1];
-            ptx::named_bar_sync(bar_id, 128);  // everyone has read gf before the leader rewrites it
+            const int valid = gf[2 * (n & 1)], trow0 = gf[2 * (n & 1) + 1];
             if (valid < 0) break;
             // each thread observes the accumulator's completion itself before
             // reading TMEM (the phase is complete, so this returns at once)
-            if (!ptx::mbar_wait_bounded(accf(e), n & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) flags[0] = 1;
+            if (!ptx::mbar_wait_bounded(accf(a), aph, watchdog, WD_OUT_MMA, kWaitLimitNs)) flags[0] = 1;
             ptx::tc_fence_after_sync();
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + e * C::ACOLS;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
             float zh, zl;
             tmem_ld_2cols(taddr + D, zh, zl);
             const float inv = __frcp_rn(zh + zl + g.eps);
@@ -909,7 +947,7 @@ __global__ void __launch_bounds__(608, 1)
                 }
             }
             ptx::tc_fence_before_sync();
-            ptx::mbar_arrive(acce(e));  // accumulator e may be overwritten
+            warp_arrive(acce(a), lane);  // accumulator a may be overwritten
             if (full_tile) {
                 ptx::fence_proxy_async_smem();
                 ptx::named_bar_sync(bar_id, 128);

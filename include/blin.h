@@ -209,6 +209,12 @@ BLIN_API blin_status blin_device_status(int *code);
  * cudaEvent_t handles, owned by the caller).  NULL turns recording off. */
 BLIN_API blin_status blin_set_timing_events(void *const *events, int n);
 
+/* Number of kernels this library has launched in this process so far (all
+ * threads and devices; a profiling aid: the difference across a region counts
+ * its launches).  A tensor-core prefill or block step launches 3 (partial
+ * states, block scan, output), the general path 4 (RoPE table first). */
+BLIN_API unsigned long long blin_launch_count(void);
+
 /* Library version string. */
 BLIN_API const char *blin_version(void);
 
