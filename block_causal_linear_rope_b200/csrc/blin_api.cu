@@ -120,11 +120,11 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
     for (int b = 0; b < g.nblk && !for_size; ++b)
         chunks += ((long long)(block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
     g.chunks_per_bh = (int)chunks;
-    // The persistent kernels keep the call's whole RoPE table in shared memory
-    // when it is small; otherwise they read it from global memory.
+    // The tensor-core kernels keep the call's whole RoPE table in shared memory;
+    // a call whose table does not fit next to their rings takes the CUDA-core path.
     const long long tab_entries = (long long)T * g.pt + (long long)Hg * g.py + (long long)Wg * g.px;
     g.tab_smem_bytes = (int)std::min<long long>(tab_entries * (long long)sizeof(float2), 1 << 30);
-    g.tab_smem = g.tab_smem_bytes <= tc_table_smem_limit() ? 1 : 0;
+    g.tab_smem = g.tab_smem_bytes <= tc_table_smem_limit(d) ? 1 : 0;
     const size_t E = (size_t)d * d + d;
     p.tab_bytes = align256(sizeof(float2) * ((size_t)T * g.pt + (size_t)Hg * g.py + (size_t)Wg * g.px + 1));
     p.part_bytes = align256(sizeof(float) * (size_t)g.BH * g.nblk * g.cpb * E);

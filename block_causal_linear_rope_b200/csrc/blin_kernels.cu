@@ -113,7 +113,12 @@ static cudaError_t set_smem(int bytes) {
     return e;
 }
 
-int tc_table_smem_limit() { return 24 * 1024; }
+// Largest RoPE table (bytes) the tensor-core kernels can hold in shared memory
+// next to their rings (227 KB per CTA).
+int tc_table_smem_limit(int d) {
+    const int fixed = d == 32 ? std::max(P1<32>::FIXED, P2<32>::FIXED) : std::max(P1<64>::FIXED, P2<64>::FIXED);
+    return std::min(24 * 1024, 227 * 1024 - fixed);
+}
 
 // Launch with programmatic dependent launch allowed: the kernel may start
 // while the previous kernel in the stream finishes; it calls
@@ -143,10 +148,12 @@ static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, i
 
 cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
                         float *z_out, cudaStream_t s) {
-    const int E4 = (d * d + d) / 4;
-    const dim3 grid((E4 + kScanSlice - 1) / kScanSlice, g.BH);
+    const long long cols = (long long)g.BH * ((d * d + d) / 4);  // (head, float4 column) pairs
+    const dim3 grid((unsigned)((cols + kScanSlice - 1) / kScanSlice));
     const int groups = g.nblk < 32 ? (g.nblk > 0 ? g.nblk : 1) : 32;  // thread groups of 32 columns
-    cudaError_t e = launch_pdl(scan_kernel, grid, dim3(kScanSlice * groups), 0, s, g, d, S_in, z_in, S_out, z_out);
+    const int seg = g.nblk < kScanSeg ? (g.nblk > 0 ? g.nblk : 1) : kScanSeg;
+    const int smem = seg * kScanSlice * (int)sizeof(float4);
+    cudaError_t e = launch_pdl(scan_kernel, grid, dim3(kScanSlice * groups), smem, s, g, d, S_in, z_in, S_out, z_out);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

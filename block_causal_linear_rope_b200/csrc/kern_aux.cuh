@@ -56,24 +56,32 @@ __global__ void rope_table_kernel(float2 *tab, int T, int t0, int Hg, int Wg, in
 // One CTA per (head, 32 float4 columns): thread groups form the block sums
 // P_b in parallel (their chunk loads all in flight), then one group runs the
 // chain over blocks from shared memory.  Blocks are taken kScanSeg at a time.
-constexpr int kScanSlice = 32;  // float4 columns per CTA
+constexpr int kScanSlice = 32;  // (head, float4 column) pairs per CTA: one per lane
 constexpr int kScanBatch = 8;   // chunk loads issued together per block
-constexpr int kScanSeg = 64;    // blocks staged in shared memory at once (32 KB)
+constexpr int kScanSeg = 64;    // blocks staged in shared memory at once (at most 32 KB)
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
+// Inclusive scan over blocks of the chunk partial states, per head, in a fixed
+// order: S_<=b = S_<=b-1 + ((c0 + c1) + c2 ...) over block b's chunks, starting
+// from the carried state (S_in, z_in) or zero.  The (head, float4 column)
+// pairs of all heads are laid end to end and each CTA takes 32 consecutive
+// ones, so no lane idles on a head's ragged last columns; thread group j of a
+// CTA sums the chunks of blocks j, j + groups, ... into shared memory and group
+// 0 then chains them.
 __global__ void __launch_bounds__(1024) scan_kernel(KGeom g, int d, const float *S_in, const float *z_in,
                                                     float *S_out, float *z_out) {
-    __shared__ float4 sm[kScanSeg * kScanSlice];
+    extern __shared__ float4 sm[];  // [min(nblk, kScanSeg)][kScanSlice]
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");  // chunk partials come from the previous kernel
     const int E4 = (d * d + d) / 4;
-    const int bh = blockIdx.y, col = threadIdx.x % kScanSlice, grp = threadIdx.x / kScanSlice;
+    const int col = threadIdx.x % kScanSlice, grp = threadIdx.x / kScanSlice;
     const int ngrp = blockDim.x / kScanSlice;
-    const int e4 = blockIdx.x * kScanSlice + col;
-    const bool live = e4 < E4;
+    const long long f = (long long)blockIdx.x * kScanSlice + col;
+    const bool live = f < (long long)g.BH * E4;
+    const int bh = live ? (int)(f / E4) : 0, e4 = live ? (int)(f - (long long)bh * E4) : 0;
     const float4 *part = reinterpret_cast<const float4 *>(g.part);
     float4 *prefix = reinterpret_cast<float4 *>(g.prefix);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -259,21 +259,24 @@ struct P1 {
     static constexpr int M = D == 32 ? 64 : 128;          // [K~^T ; phi(K)^T]
     static constexpr int N = D == 32 ? D + 8 : D + 16;   // [V | ones]
     static constexpr int NP = D == 32 ? 2 : 1;           // independent pipelines per CTA (MMA issuers)
-    static constexpr int NL = D == 32 ? 4 : 3;           // landing stages per pipeline: K | V; V is read by the MMA
+    static constexpr int NK = D == 32 ? 4 : 3;           // K landing slots per pipeline (free once read)
+    static constexpr int NV = D == 32 ? 5 : 4;           // V landing slots per pipeline (free once the MMA is done)
     static constexpr int NO = 2;                         // operand sets per pipeline: K~ | phi
     static constexpr int NACC = 2;                       // TMEM accumulators per pipeline (chunks in flight)
     static constexpr int ACOLS = D == 32 ? 64 : 128;     // TMEM columns per accumulator
     static constexpr uint32_t TCOLS = NP * NACC * ACOLS;
     static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
-    static constexpr int NBAR = 2 * NL + 2 * NO + 2 * NACC;  // mbarriers per pipeline
+    static constexpr int NBAR = 2 * NK + NV + NO + 2 * NACC;  // mbarriers per pipeline
     static constexpr int CTRL = 1024;
     static constexpr int BARS = 512;                     // mbarrier area at the start of the control block
-    static constexpr int FIXED = NP * (NL + NO) * 2 * TB + TB + CTRL + 1024;  // + RoPE table
+    static constexpr int RINGS = NP * (2 * NO + NK + NV) * TB;  // operand, K and V rings of all pipelines
+    static constexpr int FIXED = RINGS + TB + CTRL + 1024;  // + RoPE table
     static constexpr int THREADS = 32 * 6 * NP;  // warps [0, 4NP) transform, then NP producers, NP MMA issuers
     static_assert(NP * NBAR * 8 <= BARS, "mbarriers overflow their area");
-    static_assert(BARS + 4 * NP * (4 * NL + 4 * NO) + 16 <= CTRL, "control block overflow");
-    // the B operand's second N atom (the ones block) sits above every landing slot
-    static_assert(NP * (NL + NO) * 2 * TB - TB < (1 << 18), "LBO field range");
+    static_assert(BARS + 4 * NP * (4 * NK + 4 * NO) + 16 <= CTRL, "control block overflow");
+    static_assert(NV > NO, "an operand slot's release is read from the V ring's tile-done barriers");
+    // the B operand's second N atom (the ones block) sits above every V slot
+    static_assert(NP * NV * TB < (1 << 18), "LBO field range");
     static_assert(TCOLS <= 512, "TMEM holds 512 columns");
 };
 
@@ -284,50 +287,60 @@ struct P1 {
 // issuers' MMAs overlap in the tensor core.  Pipeline p takes every other
 // chunk of the CTA's static round robin (chunks j, j + grid, ..., chunk-index
 // major so the short last chunk of every block comes last and spreads evenly).
-// Per pipeline: a producer thread lands K and V tiles with TMA; four
-// transform warps read K and write the A operand (K~, phi(K)) into an operand
-// ring; an MMA thread accumulates [K~^T; phi^T] x [V | 1] into a TMEM
-// accumulator per chunk, taking V straight from the landing slot (a slot is
-// free after 5 arrivals: 4 transform warps + 1 commit).  Two tiles into the
-// next chunk, the transform warps read the finished accumulator back (each warp
-// its TMEM subpartition) and write the chunk partial to global memory.
+// Per pipeline: a producer thread lands each K tile and V tile with TMA in
+// two rings; four transform warps read K (its slot is free again at once) and
+// write the A operand (K~, phi(K)) into an operand ring; an MMA thread
+// accumulates [K~^T; phi^T] x [V | 1] into a TMEM accumulator per chunk,
+// taking V straight from its landing slot, and commits once per tile to that V
+// slot's tile-done barrier, which frees both the V slot and the tile's operand
+// slot.  Two tiles into the next chunk, the transform warps read the finished
+// accumulator back (each warp its TMEM subpartition) and write the chunk
+// partial to global memory.
 template <int D, int PT, int PY, int PX>
 __global__ void __launch_bounds__(P1<D>::THREADS, 1)
     partial_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                       KGeom g, int *watchdog) {
     using C = P1<D>;
-    constexpr int NP = C::NP, NL = C::NL, NO = C::NO, NA = C::NACC, TB = C::TB, ROWB = C::ROWB, E = D * D + D;
+    constexpr int NP = C::NP, NK = C::NK, NV = C::NV, NO = C::NO, NA = C::NACC, TB = C::TB, ROWB = C::ROWB,
+                  E = D * D + D;
     constexpr uint32_t IDESC = ptx::idesc_bf16_f32(C::M, C::N, 1, 1);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *land0 = smem;                         // [NP][NL][K | V]
-    uint8_t *opnd0 = land0 + NP * NL * 2 * TB;     // [NP][NO][K~ | phi]
-    uint8_t *ones = opnd0 + NP * NO * 2 * TB;      // constant B block (above every V tile: positive LBO)
+    uint8_t *opnd0 = smem;                         // [NP][NO][K~ | phi]
+    uint8_t *kring0 = opnd0 + NP * NO * 2 * TB;    // [NP][NK][K]
+    uint8_t *vring0 = kring0 + NP * NK * TB;       // [NP][NV][V]
+    uint8_t *ones = vring0 + NP * NV * TB;         // constant B block (above every V tile: positive LBO)
     uint8_t *ctrl = ones + TB;
     volatile int *flags = reinterpret_cast<volatile int *>(ctrl + C::BARS);  // [0] abort
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + C::BARS + 4);
-    int *info0 = reinterpret_cast<int *>(ctrl + C::BARS + 16);          // [NP][NL + NO][4]
+    int *info0 = reinterpret_cast<int *>(ctrl + C::BARS + 16);          // [NP][NK + NO][4]
     float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this thread's pipeline
     const int pipe = warp < 4 * NP ? warp >> 2 : (warp - 4 * NP) % NP;
-    uint8_t *land = land0 + pipe * NL * 2 * TB;
+    uint8_t *kring = kring0 + pipe * NK * TB;
+    uint8_t *vring = vring0 + pipe * NV * TB;
     uint8_t *opnd = opnd0 + pipe * NO * 2 * TB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl) + pipe * C::NBAR;
-    int *linfo = info0 + pipe * 4 * (NL + NO);  // [NL][4] unit, tile, valid, last
-    int *oinfo = linfo + 4 * NL;                 // [NO][4]
-    auto lk = [&](int s) { return land + s * 2 * TB; };
-    auto lv = [&](int s) { return land + s * 2 * TB + TB; };
+    int *linfo = info0 + pipe * 4 * (NK + NO);  // [NK][4] unit, tile, valid, last
+    int *oinfo = linfo + 4 * NK;                 // [NO][4]
+    auto lk = [&](int s) { return kring + s * TB; };
+    auto lv = [&](int s) { return vring + s * TB; };
     auto ok_ = [&](int s) { return opnd + s * 2 * TB; };
     auto op_ = [&](int s) { return opnd + s * 2 * TB + TB; };
-    auto lfull = [&](int s) { return ptx::smem_u32(bars + s); };
-    auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
-    auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
-    auto oempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
-    auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + a); };
-    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + 2 * NO + NA + a); };
+    // kfull[s]: K and V of the tile in K slot s have landed (TMA bytes);
+    // kempty[s]: its K has been read (4 transform warps);
+    // tdone[s]: the MMAs of the tile in V slot s are done (1 commit): V slot s
+    //   and that tile's operand slot are free;
+    // ofull[s]: operand slot s is written (4 transform warps)
+    auto kfull = [&](int s) { return ptx::smem_u32(bars + s); };
+    auto kempty = [&](int s) { return ptx::smem_u32(bars + NK + s); };
+    auto tdone = [&](int s) { return ptx::smem_u32(bars + 2 * NK + s); };
+    auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NK + NV + s); };
+    auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NK + NV + NO + a); };
+    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NK + NV + NO + NA + a); };
 
     const int units = g.cpb * g.nblk * g.BH;
     const int per_c = g.nblk * g.BH;
@@ -342,17 +355,15 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
     if (tid == 0) {
         for (int p = 0; p < NP; ++p) {
             uint64_t *pb = reinterpret_cast<uint64_t *>(ctrl) + p * C::NBAR;
-            for (int s = 0; s < NL; ++s) {
-                ptx::mbar_init(ptx::smem_u32(pb + s), 1);
-                ptx::mbar_init(ptx::smem_u32(pb + NL + s), 5);  // 4 transform warps (K read) + MMA commit (V read)
+            for (int s = 0; s < NK; ++s) {
+                ptx::mbar_init(ptx::smem_u32(pb + s), 1);            // kfull: producer (+ TMA bytes)
+                ptx::mbar_init(ptx::smem_u32(pb + NK + s), 4);       // kempty: one arrival per transform warp
             }
-            for (int s = 0; s < NO; ++s) {
-                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + s), 4);  // one arrival per transform warp
-                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + NO + s), 1);
-            }
+            for (int s = 0; s < NV; ++s) ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + s), 1);       // tdone: commit
+            for (int s = 0; s < NO; ++s) ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + s), 4);  // ofull
             for (int a = 0; a < NA; ++a) {
-                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + 2 * NO + a), 1);
-                ptx::mbar_init(ptx::smem_u32(pb + 2 * NL + 2 * NO + NA + a), 4);  // one arrival per transform warp
+                ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + NO + a), 1);       // accf: commit
+                ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + NO + NA + a), 4);  // acce: transform warps
             }
         }
         flags[0] = 0;
@@ -384,29 +395,31 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                     const int clen = min(kChunk, bntok - cs), ntiles = (clen + kTile - 1) / kTile;
                     const int row0 = bh * g.N + fb * g.HW + cs;
                     for (int t = 0; t < ntiles; ++t, ++k) {
-                        const int sl = k % NL;
-                        if (k >= NL && !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog,
-                                                               WD_PARTIAL_EMPTY, kWaitLimitNs)) {
+                        const int sk = k % NK, sv = k % NV;
+                        if ((k >= NK && !ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, watchdog,
+                                                                WD_PARTIAL_EMPTY, kWaitLimitNs)) ||
+                            (k >= NV && !ptx::mbar_wait_bounded(tdone(sv), ((k / NV) - 1) & 1, watchdog,
+                                                                WD_PARTIAL_EMPTY, kWaitLimitNs))) {
                             ok = false;
                             break;
                         }
-                        int *inf = linfo + 4 * sl;
+                        int *inf = linfo + 4 * sk;
                         inf[0] = u;
                         inf[1] = t;
                         inf[2] = min(kTile, clen - t * kTile);
                         inf[3] = t == ntiles - 1;
-                        ptx::mbar_arrive_expect_tx(lfull(sl), 2 * TB);
-                        ptx::tma_load_2d(ptx::smem_u32(lk(sl)), &mk, lfull(sl), 0, row0 + t * kTile);
-                        ptx::tma_load_2d(ptx::smem_u32(lv(sl)), &mv, lfull(sl), 0, row0 + t * kTile);
+                        ptx::mbar_arrive_expect_tx(kfull(sk), 2 * TB);
+                        ptx::tma_load_2d(ptx::smem_u32(lk(sk)), &mk, kfull(sk), 0, row0 + t * kTile);
+                        ptx::tma_load_2d(ptx::smem_u32(lv(sv)), &mv, kfull(sk), 0, row0 + t * kTile);
                     }
                 }
             }
             // end marker for the transform warps
-            const int sl = k % NL;
-            if (ok && (k < NL || ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
+            const int sk = k % NK;
+            if (ok && (k < NK || ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
                                                         kWaitLimitNs))) {
-                linfo[4 * sl] = kEndFirst;
-                ptx::mbar_arrive(lfull(sl));
+                linfo[4 * sk] = kEndFirst;
+                ptx::mbar_arrive(kfull(sk));
             }
         }
     } else if (warp >= 5 * NP) {
@@ -430,8 +443,8 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                     break;
                 }
                 ptx::tc_fence_after_sync();
-                const int sl = k % NL;  // the tile's landing slot (same tile order as the producer)
-                const uint32_t va = ptx::smem_u32(lv(sl));
+                const int sv = k % NV;  // the tile's V slot (same tile order as the producer)
+                const uint32_t va = ptx::smem_u32(lv(sv));
                 // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones.
                 // Consecutive K steps are 16 token rows (16 * ROWB bytes: ROWB in the address field).
                 const uint64_t ad = ptx::smem_desc(ptx::smem_u32(ok_(so)), TB, 8 * ROWB, C::LAYOUT);
@@ -441,8 +454,7 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                 for (int kk = 0; kk < kTile / 16; ++kk)
                     ptx::mma_bf16_ss(dacc, ad + static_cast<uint64_t>(kk * ROWB), bd + static_cast<uint64_t>(kk * ROWB),
                                      IDESC, (t > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(oempty(so));
-                ptx::mma_commit(lempty(sl));
+                ptx::mma_commit(tdone(sv));
                 if (last) {
                     ptx::mma_commit(accf(a));
                     ++nu;
@@ -500,26 +512,24 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
         int pend_u = -1, pend_a = 0, pend_ph = 0;  // finished chunk whose epilogue is still due
         int since = 0;                            // tiles pushed since that chunk's last tile
         for (int k = 0;; ++k) {
-            const int sl = k % NL, so = k % NO;
-            if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs)) {
+            const int sk = k % NK, so = k % NO;
+            if (flags[0] || !ptx::mbar_wait_bounded(kfull(sk), (k / NK) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs)) {
                 flags[0] = 1;
                 break;
             }
-            const int *inf = linfo + 4 * sl;
+            const int *inf = linfo + 4 * sk;
             const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
             const int last = ld_volatile(inf + 3);
             // read this row of K; rows past the chunk also clear their V row
             // (the MMA reads V in place: other blocks' tokens must add nothing)
             uint32_t w[D / 2], ph[D / 2];
             const bool live = u >= 0 && r < valid;
-            if (live) load_row<D>(lk(sl), r, w);
-            else if (u >= 0) zero_row<D>(lv(sl), r);
-            if (u >= 0) {
-                if (valid < kTile) ptx::fence_proxy_async_smem();
-                warp_arrive(lempty(sl), lane);
-            }
-            if (k >= NO &&
-                !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
+            if (live) load_row<D>(lk(sk), r, w);
+            else if (u >= 0) zero_row<D>(lv(k % NV), r);
+            if (u >= 0) warp_arrive(kempty(sk), lane);
+            // operand slot so was last used by tile k - NO: wait for its MMAs
+            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NV), ((k - NO) / NV) & 1, watchdog,
+                                                   WD_PARTIAL_READY, kWaitLimitNs)) {
                 flags[0] = 1;
                 break;
             }
