@@ -161,12 +161,13 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 2D map over [rows][d] bf16 rows, 128-row boxes, swizzle = row width (64 B / 128 B).
-static bool make_map(CUtensorMap *m, const void *base, long long rows, int d) {
+// 2D view [rows][d] bf16 with `box_rows`-row boxes, swizzled to the row size.
+static bool make_map(CUtensorMap *m, const void *base, long long rows, int d, int box_rows = kTile) {
     EncodeTiledFn enc = encode_fn();
     if (enc == nullptr) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)kTile};
+    cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -200,7 +201,7 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
     if (tc) {
         const long long rows = (long long)g.BH * g.N;
         if (!make_map(&mq, q, rows, d) || !make_map(&mk, k, rows, d) || !make_map(&mv, v, rows, d) ||
-            !make_map(&mo, o, rows, d))
+            !make_map(&mo, o, rows, d, 32))
             return fail(BLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
     }
     const bool bf = dt == BLIN_BF16;

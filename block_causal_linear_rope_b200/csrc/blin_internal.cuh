@@ -80,8 +80,8 @@ cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, cons
 // Shared-memory bytes the tensor-core kernels need for a RoPE table copy of
 // `entries` float2 (0 when the table is read from global memory).
 int tc_table_smem_limit(int d);
-cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo,
-                             void *o, cudaStream_t s);
+cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo, void *o,
+                             cudaStream_t s);
 
 // Device watchdog access.
 cudaError_t read_and_clear_watchdog(int *code);

@@ -199,16 +199,19 @@ cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, cons
                                                                (units + P1<64>::NP - 1) / P1<64>::NP, s, mk, mv, g, wd);
 }
 
-cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo,
-                             void *o, cudaStream_t s) {
+cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo, void *o,
+                             cudaStream_t s) {
     int *wd = watchdog_ptr();
     if (wd == nullptr) return cudaErrorInvalidDevice;
     const long long units = (long long)g.qcpb * g.nblk * g.BH;
     const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
     __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+    // a CTA runs NP pipelines, each taking every NP-th of the CTA's groups
     if (d == 32)
-        return launch_persistent<output_tc_kernel<32, 4, 6, 6>>(true, P2<32>::FIXED + tab, P2<32>::THREADS, units, s, mq, mo, g, ob, wd);
-    return launch_persistent<output_tc_kernel<64, 8, 12, 12>>(true, P2<64>::FIXED + tab, P2<64>::THREADS, units, s, mq, mo, g, ob, wd);
+        return launch_persistent<output_tc_kernel<32, 4, 6, 6>>(true, P2<32>::FIXED + tab, P2<32>::THREADS,
+                                                                (units + P2<32>::NP - 1) / P2<32>::NP, s, mq, mo, g, ob, wd);
+    return launch_persistent<output_tc_kernel<64, 8, 12, 12>>(true, P2<64>::FIXED + tab, P2<64>::THREADS,
+                                                              (units + P2<64>::NP - 1) / P2<64>::NP, s, mq, mo, g, ob, wd);
 }
 
 }  // namespace blin

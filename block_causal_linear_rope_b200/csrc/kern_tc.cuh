@@ -526,6 +526,9 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
             const bool live = u >= 0 && r < valid;
             if (live) load_row<D>(lk(sk), r, w);
             else if (u >= 0) zero_row<D>(lv(k % NV), r);
+            // the next TMA into this K slot writes through the async proxy: order
+            // this thread's generic reads of the slot before it
+            ptx::fence_proxy_async_smem();
             if (u >= 0) warp_arrive(kempty(sk), lane);
             // operand slot so was last used by tile k - NO: wait for its MMAs
             if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NV), ((k - NO) / NV) & 1, watchdog,
@@ -590,72 +593,86 @@ template <int D>
 struct P2 {
     static constexpr int ROWB = 2 * D;
     static constexpr int TB = kTile * ROWB;
-    static constexpr int NL = D == 32 ? 12 : 2;        // landing stages (Q tiles)
-    static constexpr int NO = D == 32 ? 3 : 2;         // operand sets: q~ | phi(q)
-    static constexpr int NSTG = D == 32 ? 2 : 1;       // O staging buffers per epilogue group
-    static constexpr int N = OutB<D>::N;               // num | phi.z_hi | phi.z_lo | pad
-    static constexpr int BATOM = OutB<D>::BATOM;       // one K atom of B (N rows)
+    static constexpr int NP = D == 32 ? 2 : 1;          // independent pipelines per CTA (MMA issuers)
+    static constexpr int NL = D == 32 ? 5 : 2;          // Q landing slots per pipeline
+    static constexpr int NO = 2;                        // operand sets per pipeline: q~ | phi(q)
+    static constexpr int NACC = 4;                      // TMEM accumulators per pipeline
+    static constexpr int NT = NACC > NO + 1 ? NACC : NO + 1;  // tile-done barriers per pipeline
+    static constexpr int N = OutB<D>::N;                // num | phi.z_hi | phi.z_lo | pad
+    static constexpr int BATOM = OutB<D>::BATOM;        // one K atom of B (N rows)
     static constexpr int IMG = OutB<D>::IMG;
-    static constexpr int ACOLS = D == 32 ? 64 : 128;   // TMEM columns per accumulator
-    static constexpr int NACC = 4;                     // TMEM accumulators; epilogue group e uses e, e + 2
-    static constexpr uint32_t TCOLS = NACC * ACOLS;
+    static constexpr int ACOLS = D == 32 ? 64 : 128;    // TMEM columns per accumulator
+    static constexpr uint32_t TCOLS = NP * NACC * ACOLS;
     static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
-    static constexpr int PRE = (D * D + D) * 4;        // one fp32 prefix state (S, z)
-    static constexpr int NBARS = 2 * NL + 2 * NO + 3 * NACC + 6;
-    static constexpr int INFO = (NBARS * 8 + 15) / 16 * 16;
-    static constexpr int CTRL = 1024;
-    static constexpr int FIXED = NL * TB + NO * 2 * TB + 2 * NSTG * TB + 2 * IMG + 2 * PRE + CTRL + 1024;  // + table
-    static constexpr int THREADS = 608;  // warps 0-7 transform, 8-15 epilogue, 16 producer, 17 MMA, 18 B prep
-    static_assert(INFO + 32 * NL + 32 * NO + 16 * NACC + 64 + 16 <= CTRL, "control block overflow");
+    static constexpr int PRE = (D * D + D) * 4;         // one fp32 prefix state (S, z)
+    static constexpr int NBAR = 2 * NL + NO + NT + NACC + 6;  // + pfull, pempty, bempty (2 each)
+    static constexpr int CTRL = 2048;
+    static constexpr int BARS = 512;
+    // shared memory of one pipeline, rounded up so every pipeline's swizzled
+    // tiles stay 1024-byte aligned
+    // (+ TB: each epilogue warp's 32-row O staging area for its TMA store)
+    static constexpr int PIPE = (NL * TB + NO * 2 * TB + TB + 2 * IMG + 2 * PRE + 1023) / 1024 * 1024;
+    static constexpr int FIXED = NP * PIPE + CTRL + 1024;  // + RoPE table
+    static constexpr int THREADS = 32 * 10 * NP;  // per pipeline: 4 transform, 4 epilogue, producer, MMA warps
+    static_assert(NP * NBAR * 8 <= BARS, "mbarriers overflow their area");
+    static_assert(BARS + 16 + NP * 4 * 8 * (NL + NO) <= CTRL, "control block overflow");
     static_assert(TCOLS <= 512, "TMEM holds 512 columns");
+    static_assert(PIPE % 1024 == 0, "pipelines keep 1024-byte alignment");
 };
 
-// Persistent, one CTA per SM: CTA j takes groups j, j + grid, ... of <= 8 query
-// tiles of one (head, block).  Per group the
-// producer bulk-copies the fp32 prefix state, which a B-prep warp turns into
-// the bf16 B operand (both double-buffered); per tile it lands Q in a deep ring.  Two transform groups write [R phi(q) | phi(q)] into
-// an operand ring; the MMA issuer cycles through four TMEM accumulators, and
-// epilogue group e (warps 8+4e..11+4e) takes tiles of parity e (accumulators e
-// and e + 2), so an MMA never waits on the epilogue of the tile just before it: it divides, writes
-// bf16 rows to its staging buffer and stores them with TMA (plain stores for a
-// ragged tile).
+// Persistent, one CTA per SM, NP independent pipelines (see pass 1: two
+// issuing threads keep the tensor core fed).  Pipeline p takes every other
+// group of <= 8 query tiles of one (head, block) from the CTA's static round
+// robin.  Per pipeline: a producer thread bulk-copies each group's fp32
+// prefix state and lands its Q tiles with TMA; four transform warps build the
+// group's bf16 B operand [[S, 0], [0, z_hi z_lo]] from the prefix state, then
+// write [R phi(q) | phi(q)] per tile into an operand ring; an MMA thread
+// computes [Q~ | phi(Q)] x B into one of NACC TMEM accumulators and commits
+// once per tile to a tile-done barrier (which frees the operand slot and tells
+// the epilogue the accumulator is ready); four epilogue warps divide
+// num / (phi(q).z + eps) in fp32, free the accumulator, and each stages its 32
+// bf16 rows in shared memory and stores them with its own TMA store (plain
+// stores for the warp that holds a ragged tile's edge).  `mo` views O with
+// 32-row boxes.
 template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(608, 1)
-    output_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo,
-                     KGeom g, __nv_bfloat16 *o, int *watchdog) {
+__global__ void __launch_bounds__(P2<D>::THREADS, 1)
+    output_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo, KGeom g,
+                     __nv_bfloat16 *o, int *watchdog) {
     using C = P2<D>;
-    constexpr int NL = C::NL, NO = C::NO, NSTG = C::NSTG, TB = C::TB, ROWB = C::ROWB;
+    constexpr int NP = C::NP, NL = C::NL, NO = C::NO, NA = C::NACC, NT = C::NT, TB = C::TB, ROWB = C::ROWB;
     constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, C::N, 0, 0);
+    constexpr int QG = kQTiles * kTile;  // tokens per group
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *land = smem;                        // [NL][Q]
-    uint8_t *opnd = land + NL * TB;              // [NO][q~ | phi]
-    uint8_t *stg = opnd + NO * 2 * TB;           // [2 groups][NSTG][O]
-    uint8_t *bbuf = stg + 2 * NSTG * TB;         // [2][IMG] bf16 B operand
-    uint8_t *pbuf = bbuf + 2 * C::IMG;           // [2][PRE] fp32 prefix state
-    uint8_t *ctrl = pbuf + 2 * C::PRE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl);
-    int *linfo = reinterpret_cast<int *>(ctrl + C::INFO);  // [NL][8]: unit, tile, valid, ord, row0, last
-    int *oinfo = linfo + 8 * NL;                          // [NO][8]
-    int *ainfo = oinfo + 8 * NO;                          // [NACC][4]: valid (-1 = end), row0
-    volatile int *flags = reinterpret_cast<volatile int *>(ainfo + 4 * C::NACC);  // [0] abort, [2..3] prefix slots, [4+4e..]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ainfo + 4 * C::NACC + 16);
+    uint8_t *ctrl = smem + NP * C::PIPE;
+    volatile int *flags = reinterpret_cast<volatile int *>(ctrl + C::BARS);  // [0] abort
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + C::BARS + 4);
     float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // roles: warps [0, 4NP) transform, [4NP, 8NP) epilogue, then NP producers, NP MMA issuers
+    const int pipe = warp < 8 * NP ? (warp >> 2) % NP : (warp - 8 * NP) % NP;
+    uint8_t *pb = smem + pipe * C::PIPE;
+    uint8_t *land = pb;                           // [NL][Q]
+    uint8_t *opnd = land + NL * TB;               // [NO][q~ | phi]
+    uint8_t *ostg = opnd + NO * 2 * TB;           // [4 warps][32 rows] O staging
+    uint8_t *bbuf = ostg + TB;                    // [2][IMG] bf16 B operand
+    uint8_t *pbuf = bbuf + 2 * C::IMG;            // [2][PRE] fp32 prefix state
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl) + pipe * C::NBAR;
+    int *linfo = reinterpret_cast<int *>(ctrl + C::BARS + 16) + pipe * 8 * (NL + NO);  // [NL][8]
+    int *oinfo = linfo + 8 * NL;                                                     // [NO][8]
     auto lq = [&](int s) { return land + s * TB; };
     auto oq = [&](int s) { return opnd + s * 2 * TB; };
     auto oph = [&](int s) { return opnd + s * 2 * TB + TB; };
     auto lfull = [&](int s) { return ptx::smem_u32(bars + s); };
     auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
     auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
-    auto oempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
-    constexpr int NA = C::NACC, AB = 2 * NL + 2 * NO;
-    auto accf = [&](int a) { return ptx::smem_u32(bars + AB + a); };
-    auto accp = [&](int a) { return ptx::smem_u32(bars + AB + NA + a); };
-    auto acce = [&](int a) { return ptx::smem_u32(bars + AB + 2 * NA + a); };
-    auto bfull = [&](int a) { return ptx::smem_u32(bars + AB + 3 * NA + a); };
-    auto bempty = [&](int a) { return ptx::smem_u32(bars + AB + 3 * NA + 2 + a); };
-    auto pfull = [&](int a) { return ptx::smem_u32(bars + AB + 3 * NA + 4 + a); };
+    auto tdone = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
+    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + NO + NT + a); };
+    auto pfull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + s); };
+    auto pempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + 2 + s); };
+    auto bempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + 4 + s); };
 
     const int units = g.qcpb * g.nblk * g.BH;
     const int per_q = g.nblk * g.BH;
@@ -665,27 +682,22 @@ __global__ void __launch_bounds__(608, 1)
         bh = rem / g.nblk;
         b = rem - bh * g.nblk;
     };
-    constexpr int QG = kQTiles * kTile;  // tokens per group
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < NL; ++s) {
-            ptx::mbar_init(lfull(s), 1);
-            ptx::mbar_init(lempty(s), 4);  // one arrival per transform warp
-        }
-        for (int s = 0; s < NO; ++s) {
-            ptx::mbar_init(ofull(s), 4);
-            ptx::mbar_init(oempty(s), 1);
-        }
-        for (int a = 0; a < NA; ++a) {
-            ptx::mbar_init(accf(a), 1);
-            ptx::mbar_init(accp(a), 1);
-            ptx::mbar_init(acce(a), 4);  // one arrival per epilogue warp
-        }
-        for (int a = 0; a < 2; ++a) {
-            ptx::mbar_init(bfull(a), 1);
-            ptx::mbar_init(bempty(a), 1);
-            ptx::mbar_init(pfull(a), 1);
+        for (int p = 0; p < NP; ++p) {
+            uint64_t *bp = reinterpret_cast<uint64_t *>(ctrl) + p * C::NBAR;
+            for (int s = 0; s < NL; ++s) {
+                ptx::mbar_init(ptx::smem_u32(bp + s), 1);       // lfull: producer + TMA bytes
+                ptx::mbar_init(ptx::smem_u32(bp + NL + s), 4);  // lempty: transform warps
+            }
+            for (int s = 0; s < NO; ++s) ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + s), 4);           // ofull
+            for (int s = 0; s < NT; ++s) ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + s), 1);      // tdone
+            for (int a = 0; a < NA; ++a) ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + a), 4);  // acce
+            for (int s = 0; s < 2; ++s) {
+                ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + s), 1);      // pfull: bulk copy
+                ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + 2 + s), 4);  // pempty: transform warps
+                ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + 4 + s), 1);  // bempty: commit
+            }
         }
         flags[0] = 0;
         ptx::fence_mbar_init();
@@ -697,154 +709,111 @@ __global__ void __launch_bounds__(608, 1)
     ptx::tc_fence_before_sync();
     __syncthreads();
     ptx::tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot + pipe * NA * C::ACOLS;  // this pipeline's accumulators
 
-    if (warp == 16) {
-        // ------------------------------------------------------------ TMA producer
+    // this pipeline's groups: units blockIdx.x + (pipe + NP j) * gridDim.x
+    const int u0 = blockIdx.x + pipe * gridDim.x, ustep = NP * gridDim.x;
+
+    if (warp >= 8 * NP && warp < 9 * NP) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
             ptx::tma_prefetch_map(&mq);
-            ptx::tma_prefetch_map(&mo);
             int k = 0, nu = 0;
             bool waited = false, ok = true;
-            auto issue_b = [&](int bh, int b, int ord) {
+            auto issue_prefix = [&](int bh, int b, int ord) {
                 const int sl = ord & 1;
                 if (ord >= 2 &&
-                    !ptx::mbar_wait_bounded(bempty(sl), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))
+                    !ptx::mbar_wait_bounded(pempty(sl), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))
                     return false;
                 if (!waited) {  // the prefix states are written by the scan
                     griddep_wait();
                     waited = true;
                 }
-                flags[2 + sl] = 1;
                 ptx::mbar_arrive_expect_tx(pfull(sl), C::PRE);
                 ptx::bulk_load(ptx::smem_u32(pbuf + sl * C::PRE), g.prefix + ((size_t)bh * g.nblk + b) * (D * D + D),
                                C::PRE, pfull(sl));
                 return true;
             };
-            for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {  // static round robin
+            for (int u = u0; ok && u < units; u += ustep) {
                 int bh, b, qc;
                 decode(u, bh, b, qc);
                 const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
                 const int bntok = (fe - fb) * g.HW, qs = qc * QG;
-                if (qs < bntok) {
-                    const int qlen = min(QG, bntok - qs), ntiles = (qlen + kTile - 1) / kTile;
-                    const int row0 = bh * g.N + fb * g.HW + qs;
-                    // first group: its Q tiles go out before waiting on pass 1
-                    const int early = waited ? 0 : min(ntiles, NL);
-                    if (early == 0 && !(ok = issue_b(bh, b, nu))) break;
-                    for (int t = 0; t < ntiles; ++t, ++k) {
-                        const int sl = k % NL;
-                        if (k >= NL &&
-                            !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY, kWaitLimitNs)) {
-                            ok = false;
-                            break;
-                        }
-                        int *inf = linfo + 8 * sl;
-                        inf[0] = u;
-                        inf[1] = t;
-                        inf[2] = min(kTile, qlen - t * kTile);
-                        inf[3] = nu;
-                        inf[4] = row0 + t * kTile;
-                        inf[5] = t == ntiles - 1;
-                        ptx::mbar_arrive_expect_tx(lfull(sl), TB);
-                        ptx::tma_load_2d(ptx::smem_u32(lq(sl)), &mq, lfull(sl), 0, row0 + t * kTile);
-                        if (early > 0 && t == early - 1 && !(ok = issue_b(bh, b, nu))) break;
+                if (qs >= bntok) continue;
+                const int qlen = min(QG, bntok - qs), ntiles = (qlen + kTile - 1) / kTile;
+                const int row0 = bh * g.N + fb * g.HW + qs;
+                // the first group's Q tiles go out before waiting on the scan
+                const int early = waited ? 0 : min(ntiles, NL);
+                if (early == 0 && !(ok = issue_prefix(bh, b, nu))) break;
+                for (int t = 0; t < ntiles; ++t, ++k) {
+                    const int sl = k % NL;
+                    if (k >= NL &&
+                        !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY, kWaitLimitNs)) {
+                        ok = false;
+                        break;
                     }
-                    ++nu;
+                    int *inf = linfo + 8 * sl;
+                    inf[0] = u;
+                    inf[1] = t;
+                    inf[2] = min(kTile, qlen - t * kTile);
+                    inf[3] = nu;
+                    inf[4] = fb * g.HW + qs;  // token index (within the head) of the group's first row
+                    inf[5] = t == ntiles - 1;
+                    ptx::mbar_arrive_expect_tx(lfull(sl), TB);
+                    ptx::tma_load_2d(ptx::smem_u32(lq(sl)), &mq, lfull(sl), 0, row0 + t * kTile);
+                    if (early > 0 && t == early - 1 && !(ok = issue_prefix(bh, b, nu))) break;
                 }
+                ++nu;
             }
-            for (int e = 0; ok && e < 2; ++e, ++k) {  // end markers, one per transform group
-                const int sl = k % NL;
-                if (k >= NL &&
-                    !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY, kWaitLimitNs))
-                    break;
-                linfo[8 * sl] = e == 0 ? kEndFirst : kEndSecond;
+            // end marker for the transform warps
+            const int sl = k % NL;
+            if (ok && (k < NL || ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY,
+                                                        kWaitLimitNs))) {
+                linfo[8 * sl] = kEndFirst;
                 ptx::mbar_arrive(lfull(sl));
             }
-            // end marker for the B-prep warp
-            const int sl = nu & 1;
-            if (ok && (nu < 2 || ptx::mbar_wait_bounded(bempty(sl), ((nu >> 1) - 1) & 1, watchdog, WD_OUT_BREADY,
-                                                        kWaitLimitNs))) {
-                flags[2 + sl] = -1;
-                ptx::mbar_arrive(pfull(sl));
-            }
         }
-    } else if (warp == 18) {
-        // ------------------------------------------------------------ B prep: fp32 prefix -> bf16 B operand
-        for (int ord = 0;; ++ord) {
-            const int sl = ord & 1;
-            if (flags[0] || !ptx::mbar_wait_bounded(pfull(sl), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs)) {
-                flags[0] = 1;
-                break;
-            }
-            if (flags[2 + sl] < 0) break;
-            const float *pre = reinterpret_cast<const float *>(pbuf + sl * C::PRE);
-            uint4 *dst = reinterpret_cast<uint4 *>(bbuf + sl * C::IMG);
-            for (int item = lane; item < C::IMG / 16; item += 32) dst[item] = b_operand_chunk<D>(pre, item);
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bfull(sl));
-        }
-    } else if (warp == 17) {
+    } else if (warp >= 9 * NP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            bool ok = true;
-            int k = 0;
-            for (;; ++k) {
+            for (int k = 0;; ++k) {
                 const int so = k % NO, a = k % NA;
                 if (flags[0] || !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
-                    ok = false;
+                    flags[0] = 1;
                     break;
                 }
                 const int *inf = oinfo + 8 * so;
-                const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
-                const int ord = ld_volatile(inf + 3), row0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
+                const int u = ld_volatile(inf), ord = ld_volatile(inf + 3), last = ld_volatile(inf + 5);
                 if (u < 0) break;
-                if ((k >= NA &&
-                     !ptx::mbar_wait_bounded(acce(a), ((k / NA) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs)) ||
-                    (t == 0 &&
-                     !ptx::mbar_wait_bounded(bfull(ord & 1), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))) {
-                    ok = false;
+                if (k >= NA &&
+                    !ptx::mbar_wait_bounded(acce(a), ((k / NA) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs)) {
+                    flags[0] = 1;
                     break;
                 }
                 ptx::tc_fence_after_sync();
                 const uint32_t qa = ptx::smem_u32(oq(so)), pa = ptx::smem_u32(oph(so));
                 const uint32_t ba = ptx::smem_u32(bbuf + (ord & 1) * C::IMG);
+                const uint32_t dacc = tmem + a * C::ACOLS;
 #pragma unroll
                 for (int kk = 0; kk < 2 * D / 16; ++kk) {
                     // K atom 0 = q~, K atom 1 = phi(q); +32 B per 16-element K step
                     const int atom = kk / (D / 16), j = kk % (D / 16);
                     const uint64_t ad = ptx::smem_desc((atom ? pa : qa) + 32 * j, 16, 8 * ROWB, C::LAYOUT);
                     const uint64_t bd = ptx::smem_desc(ba + atom * C::BATOM + 32 * j, 16, 8 * ROWB, C::LAYOUT);
-                    ptx::mma_bf16_ss(tmem + a * C::ACOLS, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+                    ptx::mma_bf16_ss(dacc, ad, bd, IDESC, kk > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(oempty(so));
-                ainfo[4 * a] = valid;
-                ainfo[4 * a + 1] = row0;
-                ptx::mbar_arrive(accp(a));
-                ptx::mma_commit(accf(a));
+                ptx::mma_commit(tdone(k % NT));
                 if (last) ptx::mma_commit(bempty(ord & 1));
             }
-            if (!ok) flags[0] = 1;
-            // tell both epilogue groups there is nothing more (tiles k and k + 1)
-            for (int j = 0; ok && j < 2; ++j) {
-                const int kk = k + j, a = kk % NA;
-                if (kk >= NA &&
-                    !ptx::mbar_wait_bounded(acce(a), ((kk / NA) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs))
-                    break;
-                ainfo[4 * a] = -1;
-                ptx::mbar_arrive(accp(a));
-            }
         }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ transform warps (two groups)
-        const int grp = warp >> 2, r = tid & 127;
-        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 256);
-        ptx::named_bar_sync(1, 256);
-        const int step = 2 * kTile;
-        const int dx = step % g.Wg, dy = (step / g.Wg) % g.Hg, dt = step / g.HW;
+    } else if (warp < 4 * NP) {
+        // ------------------------------------------------------------ transform warps: one row per thread
+        const int r = tid & 127;
+        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 128 * NP);
+        ptx::named_bar_sync(1, 128 * NP);
+        const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
         TokPos tp{0, 0, 0};
-        for (int k = grp;; k += 2) {
+        for (int k = 0;; ++k) {
             const int sl = k % NL, so = k % NO;
             if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_OUT_FULL, kWaitLimitNs)) {
                 flags[0] = 1;
@@ -852,30 +821,44 @@ __global__ void __launch_bounds__(608, 1)
             }
             const int *inf = linfo + 8 * sl;
             const int u = ld_volatile(inf);
-            if (u == kEndSecond) break;
             const int t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2), ord = ld_volatile(inf + 3);
-            const int row0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
+            const int tok0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
+            if (u >= 0 && t == 0) {
+                // a new group: build its B operand from the prefix state (the
+                // slot's previous group must be done with it)
+                const int bs = ord & 1;
+                if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY,
+                                                         kWaitLimitNs)) ||
+                    !ptx::mbar_wait_bounded(pfull(bs), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs)) {
+                    flags[0] = 1;
+                    break;
+                }
+                const float *pre = reinterpret_cast<const float *>(pbuf + bs * C::PRE);
+                uint4 *dst = reinterpret_cast<uint4 *>(bbuf + bs * C::IMG);
+                for (int item = r; item < C::IMG / 16; item += 128) dst[item] = b_operand_chunk<D>(pre, item);
+                ptx::fence_proxy_async_smem();  // read by the MMA (async proxy); ordered by this tile's ofull
+                warp_arrive(pempty(bs), lane);
+            }
             uint32_t w[D / 2], ph[D / 2];
             const bool live = u >= 0 && r < valid;
             if (live) load_row<D>(lq(sl), r, w);
+            // the next TMA into this slot writes through the async proxy: order
+            // this thread's generic reads of the slot before it
+            ptx::fence_proxy_async_smem();
             if (u >= 0) warp_arrive(lempty(sl), lane);  // landing slot read
-            if (k >= NO &&
-                !ptx::mbar_wait_bounded(oempty(so), ((k / NO) - 1) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
+            // operand slot so was last used by tile k - NO: wait for its MMAs
+            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NT), ((k - NO) / NT) & 1, watchdog, WD_OUT_READY,
+                                                   kWaitLimitNs)) {
                 flags[0] = 1;
                 break;
             }
-            if (u == kEndFirst) {  // pass the end on to the MMA issuer, in operand order
+            if (u < 0) {  // pass the end on to the MMA issuer, in operand order
                 if (r == 0) oinfo[8 * so] = kEndFirst;
                 warp_arrive(ofull(so), lane);
                 break;
             }
-            if (t <= 1) {
-                int bh, b, qc;
-                decode(u, bh, b, qc);
-                tp.init(g, block_frame_begin(g, b) * g.HW + qc * QG + t * kTile + r);
-            } else {
-                tp.advance(g, dx, dy, dt);
-            }
+            if (t == 0) tp.init(g, tok0 + r);
+            else tp.advance(g, dx, dy, dt);
             if (live) {
                 phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
                 store_row<D>(oq(so), r, w);
@@ -889,91 +872,72 @@ __global__ void __launch_bounds__(608, 1)
                 int *oi = oinfo + 8 * so;
                 oi[0] = u;
                 oi[1] = t;
-                oi[2] = valid;
                 oi[3] = ord;
-                oi[4] = row0;
                 oi[5] = last;
             }
             warp_arrive(ofull(so), lane);
         }
     } else {
-        // ------------------------------------------------------------ epilogue groups (warps 8-15)
-        const int e = (warp - 8) >> 2, sub = warp & 3, er = (tid - 256) & 127;
-        const int r = 32 * sub + lane;  // tile row read back by this thread (TMEM subpartition)
-        volatile int *gf = flags + 4 + 4 * e;
-        const uint32_t bar_id = 2 + e;
-        for (int n = 0;; ++n) {  // this group's n-th tile is tile k = 2n + e, in accumulator k % NACC
-            const int a = (2 * n + e) % NA, aph = ((2 * n + e) / NA) & 1;
-            if (er == 0) {  // one thread waits and decides for the group (named barrier below)
-                int valid = -1;
-                if (!flags[0] && ptx::mbar_wait_bounded(accp(a), aph, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
-                    valid = ld_volatile(ainfo + 4 * a);
-                    gf[2 * (n & 1) + 1] = ld_volatile(ainfo + 4 * a + 1);
-                    if (valid >= 0 &&
-                        !ptx::mbar_wait_bounded(accf(a), aph, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
-                        valid = -1;
-                        flags[0] = 1;
-                    }
-                } else {
+        // ------------------------------------------------------------ epilogue warps: one row per thread
+        const int sub = warp & 3, r = 32 * sub + lane;  // tile row = this warp's TMEM subpartition lane
+        uint8_t *stg = ostg + sub * 32 * ROWB;           // this warp's 32 staged rows (swizzled like `mo`)
+        if (lane == 0) ptx::tma_prefetch_map(&mo);
+        int k = 0;
+        for (int u = u0; u < units && !flags[0]; u += ustep) {  // the producer's tile sequence
+            int bh, b, qc;
+            decode(u, bh, b, qc);
+            const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
+            const int bntok = (fe - fb) * g.HW, qs = qc * QG;
+            if (qs >= bntok) continue;
+            const int qlen = min(QG, bntok - qs), ntiles = (qlen + kTile - 1) / kTile;
+            const int row0 = bh * g.N + fb * g.HW + qs;
+            for (int t = 0; t < ntiles; ++t, ++k) {
+                const int a = k % NA;
+                if (!ptx::mbar_wait_bounded(tdone(k % NT), (k / NT) & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
                     flags[0] = 1;
+                    break;
                 }
-                gf[2 * (n & 1)] = valid;
-                // the staging buffer about to be reused has been read by its TMA store
-                ptx::bulk_wait_group_read<NSTG - 1>();
-            }
-            // the record alternates between two slots, so one barrier suffices:
-            // the leader rewrites slot n & 1 only after barrier n + 1
-            ptx::named_bar_sync(bar_id, 128);
-            const int valid = gf[2 * (n & 1)], trow0 = gf[2 * (n & 1) + 1];
-            if (valid < 0) break;
-            // each thread observes the accumulator's completion itself before
-            // reading TMEM (the phase is complete, so this returns at once)
-            if (!ptx::mbar_wait_bounded(accf(a), aph, watchdog, WD_OUT_MMA, kWaitLimitNs)) flags[0] = 1;
-            ptx::tc_fence_after_sync();
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
-            float zh, zl;
-            tmem_ld_2cols(taddr + D, zh, zl);
-            const float inv = __frcp_rn(zh + zl + g.eps);
-            const bool full_tile = valid == kTile;
-            uint8_t *st = stg + (e * NSTG + (n % NSTG)) * TB;
+                ptx::tc_fence_after_sync();
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
+                float zh, zl;
+                tmem_ld_2cols(taddr + D, zh, zl);
+                const float inv = __frcp_rn(zh + zl + g.eps);
+                uint32_t ow[D / 2];
 #pragma unroll
-            for (int half = 0; half < D / 32; ++half) {
-                float v[32];
-                ptx::tmem_ld_32cols(taddr + 32 * half, v);
-                uint32_t ow[16];
+                for (int half = 0; half < D / 32; ++half) {
+                    float v[32];
+                    ptx::tmem_ld_32cols(taddr + 32 * half, v);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) ow[q] = pack_bf16x2(v[2 * q] * inv, v[2 * q + 1] * inv);
-                if (r < valid) {
-                    if (full_tile) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            *reinterpret_cast<uint4 *>(st + swz_chunk<D>(r, 4 * half + j)) =
-                                make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)trow0 + r) * D + 32 * half);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
+                    for (int q = 0; q < 16; ++q) ow[16 * half + q] = pack_bf16x2(v[2 * q] * inv, v[2 * q + 1] * inv);
+                }
+                ptx::tc_fence_before_sync();
+                warp_arrive(acce(a), lane);  // the accumulator is read: the MMA may overwrite it
+                const int valid = min(kTile, qlen - t * kTile);
+                if (32 * sub + 32 <= valid) {
+                    // whole warp in range: stage the 32 rows and store them with TMA
+                    if (lane == 0) ptx::bulk_wait_group_read<0>();  // the previous store has read the staging
+                    __syncwarp();
+                    store_row<D>(stg, lane, ow);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::tma_store_2d(&mo, ptx::smem_u32(stg), 0, row0 + t * kTile + 32 * sub);
+                        ptx::bulk_commit_group();
                     }
-                }
-            }
-            ptx::tc_fence_before_sync();
-            warp_arrive(acce(a), lane);  // accumulator a may be overwritten
-            if (full_tile) {
-                ptx::fence_proxy_async_smem();
-                ptx::named_bar_sync(bar_id, 128);
-                if (er == 0) {
-                    ptx::tma_store_2d(&mo, ptx::smem_u32(st), 0, trow0);
-                    ptx::bulk_commit_group();
+                } else if (r < valid) {  // a ragged tile's edge: plain stores of the valid rows
+                    uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)row0 + t * kTile + r) * D);
+#pragma unroll
+                    for (int j = 0; j < D / 8; ++j) dst[j] = make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
                 }
             }
         }
-        if (er == 0) ptx::bulk_wait_group<0>();
+        if (lane == 0) ptx::bulk_wait_group<0>();  // stores complete before the CTA exits
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(tmem, C::TCOLS);
+        ptx::tmem_dealloc(*tmem_slot, C::TCOLS);
     }
 }
 
