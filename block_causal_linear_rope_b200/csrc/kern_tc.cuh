@@ -594,7 +594,7 @@ struct P2 {
     static constexpr int ROWB = 2 * D;
     static constexpr int TB = kTile * ROWB;
     static constexpr int NP = D == 32 ? 2 : 1;          // independent pipelines per CTA (MMA issuers)
-    static constexpr int NL = D == 32 ? 5 : 2;          // Q landing slots per pipeline
+    static constexpr int NL = D == 32 ? 6 : 3;          // Q landing slots per pipeline
     static constexpr int NO = 2;                        // operand sets per pipeline: q~ | phi(q)
     static constexpr int NACC = 4;                      // TMEM accumulators per pipeline
     static constexpr int NT = NACC > NO + 1 ? NACC : NO + 1;  // tile-done barriers per pipeline
@@ -611,7 +611,9 @@ struct P2 {
     // shared memory of one pipeline, rounded up so every pipeline's swizzled
     // tiles stay 1024-byte aligned
     // (+ TB: each epilogue warp's 32-row O staging area for its TMA store)
-    static constexpr int PIPE = (NL * TB + NO * 2 * TB + TB + 2 * IMG + 2 * PRE + 1023) / 1024 * 1024;
+    // (the fp32 prefix state is single-buffered: it is turned into the
+    // double-buffered bf16 B operand as soon as it lands)
+    static constexpr int PIPE = (NL * TB + NO * 2 * TB + TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
     static constexpr int FIXED = NP * PIPE + CTRL + 1024;  // + RoPE table
     static constexpr int THREADS = 32 * 10 * NP;  // per pipeline: 4 transform, 4 epilogue, producer, MMA warps
     static_assert(NP * NBAR * 8 <= BARS, "mbarriers overflow their area");
@@ -658,7 +660,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
     uint8_t *opnd = land + NL * TB;               // [NO][q~ | phi]
     uint8_t *ostg = opnd + NO * 2 * TB;           // [4 warps][32 rows] O staging
     uint8_t *bbuf = ostg + TB;                    // [2][IMG] bf16 B operand
-    uint8_t *pbuf = bbuf + 2 * C::IMG;            // [2][PRE] fp32 prefix state
+    uint8_t *pbuf = bbuf + 2 * C::IMG;            // [PRE] fp32 prefix state
     uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl) + pipe * C::NBAR;
     int *linfo = reinterpret_cast<int *>(ctrl + C::BARS + 16) + pipe * 8 * (NL + NO);  // [NL][8]
     int *oinfo = linfo + 8 * NL;                                                     // [NO][8]
@@ -721,17 +723,17 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
             int k = 0, nu = 0;
             bool waited = false, ok = true;
             auto issue_prefix = [&](int bh, int b, int ord) {
-                const int sl = ord & 1;
-                if (ord >= 2 &&
-                    !ptx::mbar_wait_bounded(pempty(sl), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))
+                // the previous group's prefix has been turned into its B operand
+                if (ord >= 1 &&
+                    !ptx::mbar_wait_bounded(pempty(0), (ord - 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))
                     return false;
                 if (!waited) {  // the prefix states are written by the scan
                     griddep_wait();
                     waited = true;
                 }
-                ptx::mbar_arrive_expect_tx(pfull(sl), C::PRE);
-                ptx::bulk_load(ptx::smem_u32(pbuf + sl * C::PRE), g.prefix + ((size_t)bh * g.nblk + b) * (D * D + D),
-                               C::PRE, pfull(sl));
+                ptx::mbar_arrive_expect_tx(pfull(0), C::PRE);
+                ptx::bulk_load(ptx::smem_u32(pbuf), g.prefix + ((size_t)bh * g.nblk + b) * (D * D + D), C::PRE,
+                               pfull(0));
                 return true;
             };
             for (int u = u0; ok && u < units; u += ustep) {
@@ -829,15 +831,15 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
                 const int bs = ord & 1;
                 if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY,
                                                          kWaitLimitNs)) ||
-                    !ptx::mbar_wait_bounded(pfull(bs), (ord >> 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs)) {
+                    !ptx::mbar_wait_bounded(pfull(0), ord & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs)) {
                     flags[0] = 1;
                     break;
                 }
-                const float *pre = reinterpret_cast<const float *>(pbuf + bs * C::PRE);
+                const float *pre = reinterpret_cast<const float *>(pbuf);
                 uint4 *dst = reinterpret_cast<uint4 *>(bbuf + bs * C::IMG);
                 for (int item = r; item < C::IMG / 16; item += 128) dst[item] = b_operand_chunk<D>(pre, item);
                 ptx::fence_proxy_async_smem();  // read by the MMA (async proxy); ordered by this tile's ofull
-                warp_arrive(pempty(bs), lane);
+                warp_arrive(pempty(0), lane);
             }
             uint32_t w[D / 2], ph[D / 2];
             const bool live = u >= 0 && r < valid;
