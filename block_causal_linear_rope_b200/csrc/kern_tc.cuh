@@ -1,31 +1,21 @@
 // Tensor-core path for bf16 Q/K/V on sm_100a (d = 32 or 64).
 //
-// Pass 1, partial_tc_kernel: one CTA per state chunk (<= 1024 tokens of one
-//   block of one head).  A producer warp streams 128-token K and V tiles into
-//   shared memory with TMA (64B/128B swizzle).  Four transform warps overwrite
-//   each K row in place with R_m phi(k_m) (bf16) and, for d = 32, also write
-//   phi(k_m) into a second tile.  One MMA thread accumulates
+// Pass 1, partial_tc_kernel: per chunk (<= 1024 tokens of one block of one
+//   head) the partial states P = sum (R_m phi(k_m)) v_m^T and zp = sum phi(k_m)
+//   from one contraction
 //       [K~^T ; phi(K)^T] x [V | 1]      (tcgen05.mma, fp32 in TMEM)
-//   so the d x d block state P = K~^T V and the denominator state
-//   zp = sum phi(k) come out of one contraction; both operands are MN-major
-//   views of the token-major tiles.  For d = 64 the tensor core computes P and
-//   the transform warps sum zp in fp32 registers.  The transform warps then
-//   write the chunk's partial state; the last chunk of each head to finish
-//   (atomic counter, no waiting) runs the fixed-order inclusive scan over
-//   blocks for that head.
-// Pass 2, output_tc_kernel: one CTA per group of <= 8 query tiles of one block
-//   of one head.  Epilogue warps first turn S_<=b, z_<=b into a bf16 B operand
-//       [[S, 0], [0, z_hi z_lo]]   (K = 2d rows, N = d + 16 columns)
-//   A producer warp streams Q tiles; transform warps write [R phi(q) | phi(q)]
-//   as the bf16 A operand; one MMA thread computes
-//       [Q~ | phi(Q)] x B = [num | phi(q).z_hi | phi(q).z_lo]
-//   into one of two TMEM accumulators; epilogue warps read it back, form
-//   o = num / (phi(q).z + eps) in fp32, write bf16 rows in place over the Q
-//   tile and store them with TMA (plain stores for a ragged last tile).
+//   whose operands are MN-major views of the token-major tiles.
+// Pass 2, output_tc_kernel: per group of <= 8 query tiles of one block of one
+//   head, numerator and denominator from one contraction
+//       [Q~ | phi(Q)] x [[S, 0], [0, z_hi z_lo]] = [num | phi(q).z_hi | phi(q).z_lo]
+//   then o = num / (phi(q).z + eps) in fp32, stored as bf16.
 //
-// Roles hand tiles to each other through mbarriers only (no CTA-wide barrier
-// inside the main loops) and every wait is bounded (ptx::mbar_wait_bounded).
-// Grids are ordered chunk-index-major so the short last chunks run last.
+// Both kernels are persistent (one CTA per SM) and split into roles (TMA
+// producer, transform warps, one MMA-issuing thread, epilogue) that hand tiles
+// to each other through mbarrier rings only; each CTA runs two such pipelines
+// at d = 32 (see the pass 1 comment for why).  Every wait is bounded
+// (ptx::mbar_wait_bounded), and work is ordered chunk-index major so the
+// short last chunks of every block run last.
 #pragma once
 
 #include <cuda_bf16.h>
