@@ -132,10 +132,13 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
     return p;
 }
 
-static size_t plan_bytes(const Plan &p) { return 256 + p.tab_bytes + p.part_bytes + p.prefix_bytes; }
+// 256 bytes of alignment slack, 256 for the work counters, then the tables and states
+static size_t plan_bytes(const Plan &p) { return 512 + p.tab_bytes + p.part_bytes + p.prefix_bytes; }
 
 static void plan_bind(Plan &p, void *ws) {
     uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255);
+    p.g.sched = reinterpret_cast<unsigned int *>(base);
+    base += 256;
     p.g.tab = reinterpret_cast<const float2 *>(base);
     p.g.part = reinterpret_cast<float *>(base + p.tab_bytes);
     p.g.prefix = reinterpret_cast<float *>(base + p.tab_bytes + p.part_bytes);
@@ -213,6 +216,9 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
         g_launches.fetch_add(1, std::memory_order_relaxed);
     }
     mark(0, true, s);
+    // the tensor-core passes hand out work units through counters that start at zero
+    if (tc && (e = cudaMemsetAsync(g.sched, 0, 4 * sizeof(unsigned int), s)) != cudaSuccess)
+        return cuda_fail(e, "work counter reset");
     mark(1, false, s);
     e = tc ? launch_partial_tc(g, d, mk, mv, s) : launch_partial_simt(g, d, bf, k, v, s);
     if (e != cudaSuccess) return cuda_fail(e, "partial-state launch");

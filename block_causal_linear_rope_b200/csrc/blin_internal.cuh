@@ -32,6 +32,7 @@ struct KGeom {
     int tab_y, tab_x;     // offsets (in float2) of the y and x tables
     float *part;          // [BH][nblk][cpb][d*d + d] chunk partial states
     float *prefix;        // [BH][nblk][d*d + d] inclusive prefix states S_<=b, z_<=b
+    unsigned int *sched;  // [4] work counters for dynamic scheduling, zeroed before each call
     int chunks_per_bh;    // state chunks of one head in this call
     double theta;         // RoPE base
     int tab_smem;         // 1: the RoPE table fits the tensor-core kernels' shared memory

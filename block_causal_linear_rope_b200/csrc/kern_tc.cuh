@@ -274,9 +274,10 @@ struct P1 {
 // The CTA runs NP independent pipelines, so that NP threads issue MMAs: one
 // thread issues a tcgen05.mma about every 50 cycles and the eight M = 64 MMAs
 // a 128-token tile needs from one thread would not keep up with HBM, while two
-// issuers' MMAs overlap in the tensor core.  Pipeline p takes every other
-// chunk of the CTA's static round robin (chunks j, j + grid, ..., chunk-index
-// major so the short last chunk of every block comes last and spreads evenly).
+// issuers' MMAs overlap in the tensor core.  Chunks are taken in
+// chunk-index-major order (the short last chunk of every block comes last):
+// pipeline p of CTA j first takes chunk j + p * grid, then the next unclaimed
+// chunk from a work counter, so all pipelines finish within about one chunk.
 // Per pipeline: a producer thread lands each K tile and V tile with TMA in
 // two rings; four transform warps read K (its slot is free again at once) and
 // write the A operand (K~, phi(K)) into an operand ring; an MMA thread
@@ -376,7 +377,15 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
             ptx::tma_prefetch_map(&mv);
             int k = 0;
             bool ok = true;
-            for (int u = blockIdx.x + pipe * gridDim.x; ok && u < units; u += NP * gridDim.x) {  // static round robin
+            // the first NP * grid chunks are dealt out statically (chunk blockIdx.x + pipe * grid); after
+            // that each pipeline takes the next unclaimed chunk from a counter, in chunk-index-major
+            // order, so the long chunks go first and every pipeline ends within about one chunk of the
+            // others.  The claim for the following chunk is issued a chunk ahead (its latency hidden).
+            const int first_dyn = NP * gridDim.x;
+            int next = first_dyn + static_cast<int>(atomicAdd(g.sched, 1u));
+            for (int u = blockIdx.x + pipe * gridDim.x; ok && u < units;) {
+                const int u_next = next;
+                if (u_next < units) next = first_dyn + static_cast<int>(atomicAdd(g.sched, 1u));
                 int bh, b, c;
                 decode(u, bh, b, c);
                 const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
@@ -403,6 +412,7 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                         ptx::tma_load_2d(ptx::smem_u32(lv(sv)), &mv, kfull(sk), 0, row0 + t * kTile);
                     }
                 }
+                u = u_next;
             }
             // end marker for the transform warps
             const int sk = k % NK;

@@ -54,15 +54,15 @@ def ws(B, H, d, g):
 
 
 def test_workspace_size_formula():
-    # RoPE table + chunk partials + prefix states, each padded to 256 B, plus
-    # 256 B of alignment slack
+    # work counters (256 B) + RoPE table + chunk partials + prefix states, each
+    # padded to 256 B, plus 256 B of alignment slack
     B, H, d = 1, 70, 32
     g = geom()
     E = d * d + d
     nblk = 21 // 3 + 1
     cpb = -(-(3 * 30 * 52) // 1024)
     pad = lambda x: (x + 255) // 256 * 256
-    want = 256 + pad(8 * (21 * 4 + 30 * 6 + 52 * 6 + 1)) + pad(4 * B * H * nblk * cpb * E) + pad(4 * B * H * nblk * E)
+    want = 512 + pad(8 * (21 * 4 + 30 * 6 + 52 * 6 + 1)) + pad(4 * B * H * nblk * cpb * E) + pad(4 * B * H * nblk * E)
     assert ws(B, H, d, g) == want
 
 
