@@ -375,6 +375,7 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
         if (lane == 0) {
             ptx::tma_prefetch_map(&mk);
             ptx::tma_prefetch_map(&mv);
+            const uint64_t stream_policy = ptx::l2_evict_first();  // K and V are read once
             int k = 0;
             bool ok = true;
             // the first NP * grid chunks are dealt out statically (chunk blockIdx.x + pipe * grid); after
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                         inf[2] = min(kTile, clen - t * kTile);
                         inf[3] = t == ntiles - 1;
                         ptx::mbar_arrive_expect_tx(kfull(sk), 2 * TB);
-                        ptx::tma_load_2d(ptx::smem_u32(lk(sk)), &mk, kfull(sk), 0, row0 + t * kTile);
-                        ptx::tma_load_2d(ptx::smem_u32(lv(sv)), &mv, kfull(sk), 0, row0 + t * kTile);
+                        ptx::tma_load_2d_hint(ptx::smem_u32(lk(sk)), &mk, kfull(sk), 0, row0 + t * kTile, stream_policy);
+                        ptx::tma_load_2d_hint(ptx::smem_u32(lv(sv)), &mv, kfull(sk), 0, row0 + t * kTile, stream_policy);
                     }
                 }
                 u = u_next;
@@ -720,6 +721,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             ptx::tma_prefetch_map(&mq);
+            const uint64_t stream_policy = ptx::l2_evict_first();  // Q is read once
             int k = 0, nu = 0;
             bool waited = false, ok = true;
             auto issue_prefix = [&](int bh, int b, int ord) {
@@ -762,7 +764,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
                     inf[4] = fb * g.HW + qs;  // token index (within the head) of the group's first row
                     inf[5] = t == ntiles - 1;
                     ptx::mbar_arrive_expect_tx(lfull(sl), TB);
-                    ptx::tma_load_2d(ptx::smem_u32(lq(sl)), &mq, lfull(sl), 0, row0 + t * kTile);
+                    ptx::tma_load_2d_hint(ptx::smem_u32(lq(sl)), &mq, lfull(sl), 0, row0 + t * kTile, stream_policy);
                     if (early > 0 && t == early - 1 && !(ok = issue_prefix(bh, b, nu))) break;
                 }
                 ++nu;
@@ -884,6 +886,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
         const int sub = warp & 3, r = 32 * sub + lane;  // tile row = this warp's TMEM subpartition lane
         uint8_t *stg = ostg + sub * 32 * ROWB;           // this warp's 32 staged rows (swizzled like `mo`)
         if (lane == 0) ptx::tma_prefetch_map(&mo);
+        const uint64_t stream_policy = ptx::l2_evict_first();  // O is written once
         int k = 0;
         for (int u = u0; u < units && !flags[0]; u += ustep) {  // the producer's tile sequence
             int bh, b, qc;
@@ -923,7 +926,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        ptx::tma_store_2d(&mo, ptx::smem_u32(stg), 0, row0 + t * kTile + 32 * sub);
+                        ptx::tma_store_2d_hint(&mo, ptx::smem_u32(stg), 0, row0 + t * kTile + 32 * sub, stream_policy);
                         ptx::bulk_commit_group();
                     }
                 } else if (r < valid) {  // a ragged tile's edge: plain stores of the valid rows
