@@ -201,14 +201,19 @@ def barrier(world: int):
 
 
 # ----------------------------------------------------------------------------- oracle timing
-def oracle_sample(w: workloads.Workload, q, k, v, rows_total: int, seed: int = 0):
-    """Time the explicit pair-sum oracle on `rows_total` seeded query rows (all heads)."""
+def oracle_sample(w: workloads.Workload, q, k, v, rows_total: int, seed: int = 0, heads: int = 0):
+    """Time the explicit pair-sum oracle on `rows_total` seeded query rows of `heads` seeded heads
+    (0: all heads); returns (token*heads per second, seconds)."""
     import oracle
     pos, blk = oracle.grid(w.T, w.Hg, w.Wg, w.F)
-    rows = np.sort(np.random.default_rng([seed, 5]).choice(w.N, size=rows_total, replace=False))
+    rng = np.random.default_rng([seed, 5])
+    rows = np.sort(rng.choice(w.N, size=rows_total, replace=False))
     qs = q.reshape(-1, w.N, w.d)
     ks = k.reshape(-1, w.N, w.d)
     vs = v.reshape(-1, w.N, w.d)
+    if 0 < heads < qs.shape[0]:
+        hsel = np.sort(rng.choice(qs.shape[0], size=heads, replace=False))
+        qs, ks, vs = qs[hsel], ks[hsel], vs[hsel]
     t0 = time.perf_counter()
     oracle.attention_rows(qs, ks, vs, pos, blk, rows, w.split, w.theta, w.eps)
     dt = time.perf_counter() - t0
@@ -226,16 +231,19 @@ def run_reference(args, w):
     if world > 1 and rank != 0:
         return
     q, k, v = workloads.call_tensors(w)
-    rows = args.ref_rows
-    for _ in range(args.warmup):
-        oracle_sample(w, q, k, v, rows, seed=1)
+    # A bounded sample per step: one seeded query row per core (the oracle parallelises over
+    # rows) of a seeded subset of heads, sized so the whole run stays near a minute whatever K is.
+    rows = args.ref_rows or omp_threads()
+    heads = max(1, min(w.B * w.H, 7000 // max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample(w, q, k, v, rows, seed=1 + i, heads=heads)
     times = []
     for i in range(args.steps):
-        _, dt = oracle_sample(w, q, k, v, rows, seed=100 + i)
+        _, dt = oracle_sample(w, q, k, v, rows, seed=100 + i, heads=heads)
         times.append(dt)
     per_step = sum(times) / len(times)
-    value = rows * w.B * w.H / per_step
-    sample = (f"{rows} seeded query rows x {w.B * w.H} heads of the {w.name} workload per step, "
+    value = rows * heads / per_step
+    sample = (f"{rows} seeded query rows x {heads} seeded heads of the {w.name} workload per step, "
               f"explicit O(N^2) float64 pair sum (all keys each row may see)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
@@ -505,7 +513,8 @@ def main():
     ap.add_argument("--impl", default="blin", choices=["blin", "reference"])
     ap.add_argument("--config", default="480p", choices=["480p", "720p", "wide", "decode"])
     ap.add_argument("--cpu-rows", type=int, default=2000, help="oracle rows for the CPU baseline (about 10 s)")
-    ap.add_argument("--ref-rows", type=int, default=24, help="oracle rows per reference-arm step")
+    ap.add_argument("--ref-rows", type=int, default=None,
+                    help="oracle rows per reference-arm step (default: sized so the whole run stays near a minute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     w = workloads.CONFIGS[args.config]
