@@ -343,16 +343,57 @@ def run_blin(args, w):
     if status != 0:
         raise SystemExit(f"kernel watchdog fired (code {status})")
 
-    # ---- end to end through the C ABI: pinned host inputs in, host output back
+    # ---- end to end through the C ABI: pinned host inputs in, host output back.  Heads are
+    # independent and contiguous ([B*H][N][d]), so the step is cut into head chunks that flow
+    # through three streams (copy in, compute, copy out): one blin_prefill per chunk, and the
+    # host-to-device and device-to-host copies overlap each other and the kernels.
     h2d = 3 * qh.numel() * qh.element_size()
     d2h = oh.numel() * oh.element_size()
+    od_ref = od.clone()  # the device-resident steps' output
+    BH = w.B * w.H
+    nchunk = min(BH, args.e2e_chunks)
+    bounds = [BH * i // nchunk for i in range(nchunk + 1)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    rows = lambda x: x.view(BH, w.N, w.d)
+    qh3, kh3, vh3, oh3 = rows(qh), rows(kh), rows(vh), rows(oh)
+    qd3, kd3, vd3, od3 = rows(qd), rows(kd), rows(vd), rows(od)
+    ws_chunk = torch.empty(max(blin.workspace_size(1, bounds[i + 1] - bounds[i], w.d, grid, w.F, w.split, w.theta,
+                                                   w.eps) for i in range(nchunk)), dtype=torch.uint8, device="cuda")
+    chunk_args = []
+    for i in range(nchunk):
+        h0, h1 = bounds[i], bounds[i + 1]
+        chunk_args.append((ctypes.c_void_p(qd3[h0].data_ptr()), ctypes.c_void_p(kd3[h0].data_ptr()),
+                           ctypes.c_void_p(vd3[h0].data_ptr()), ctypes.c_void_p(od3[h0].data_ptr()),
+                           blin.BF16 if w.dtype == "bf16" else blin.F32, 1, h1 - h0, w.d, ctypes.byref(geom), None,
+                           ctypes.c_void_p(ws_chunk.data_ptr()), ws_chunk.numel(),
+                           ctypes.c_void_p(s_cmp.cuda_stream)))
+    ev_in = [torch.cuda.Event() for _ in range(nchunk)]
+    ev_cmp = [torch.cuda.Event() for _ in range(nchunk)]
+    ev_out = torch.cuda.Event()
 
     def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        step()
-        oh.copy_(od, non_blocking=True)
+        cur = torch.cuda.current_stream()
+        for s_ in (s_in, s_cmp, s_out):
+            s_.wait_stream(cur)
+        for i in range(nchunk):
+            h0, h1 = bounds[i], bounds[i + 1]
+            with torch.cuda.stream(s_in):
+                qd3[h0:h1].copy_(qh3[h0:h1], non_blocking=True)
+                kd3[h0:h1].copy_(kh3[h0:h1], non_blocking=True)
+                vd3[h0:h1].copy_(vh3[h0:h1], non_blocking=True)
+                ev_in[i].record(s_in)
+            s_cmp.wait_event(ev_in[i])
+            rc = prefill_c(*chunk_args[i])
+            if rc != 0:
+                raise RuntimeError(blin.lib.blin_last_error().decode())
+            ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                oh3[h0:h1].copy_(od3[h0:h1], non_blocking=True)
+        ev_out.record(s_out)
+        cur.wait_event(ev_out)
+        cur.wait_stream(s_in)
+        cur.wait_stream(s_cmp)
 
     for _ in range(2):
         e2e_step()
@@ -366,6 +407,9 @@ def run_blin(args, w):
     e_end.record()
     torch.cuda.synchronize()
     e_ms = max_over_ranks(e_start.elapsed_time(e_end) / e_steps, world)
+    # the chunked output must equal the one-call output (same kernels, same inputs, heads independent)
+    if not torch.equal(oh.to("cuda"), od_ref):
+        raise SystemExit("end-to-end output differs from the device-resident step")
 
     units = w.B * w.H * w.N  # token*heads per GPU per step
     value = job_throughput(units, world, ms)
@@ -392,7 +436,7 @@ def run_blin(args, w):
                      "traffic": recorded_traffic(dom, w.name),
                      "algorithmic_bytes_per_launch": alg[dom]},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e_ms},
+                "ms_per_step": e_ms, "head_chunks": nchunk},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
@@ -470,6 +514,39 @@ def run_decode(args, w):
         torch.cuda.synchronize()
         clk.timed(t_wall, time.time())
         time.sleep(0.25)
+    # host time to enqueue one block (plan, tensor maps, launches): with the GPU this fast, the
+    # stream-launched latency above is set by it
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    sequence()
+    host_us = (time.perf_counter() - t0) / nb * 1e6
+    torch.cuda.synchronize()
+    # the same nb calls captured once in a CUDA graph and replayed: per-block device time
+    # without host launch overhead
+    graph_us, graph_err = None, None
+    try:
+        cg = torch.cuda.CUDAGraph()
+        st.reset()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(cg):
+            cs = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+            for a in cargs:
+                rc = step_c(*(a[:-1] + (cs,)))
+                if rc != 0:
+                    raise RuntimeError(blin.lib.blin_last_error().decode())
+        for _ in range(2):
+            cg.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(reps):
+            cg.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        graph_us = g0.elapsed_time(g1) * 1e3 / (reps * nb)
+        del cg
+    except Exception as exc:  # capture unsupported: report why, keep the stream numbers
+        graph_err = str(exc).splitlines()[0][:200]
     status = blin.device_status()
     if status != 0:
         raise SystemExit(f"kernel watchdog fired (code {status})")
@@ -490,7 +567,9 @@ def run_decode(args, w):
                                f"{w.dtype}, commit=1, per-block latency from CUDA events around each call; "
                                f"{len(distinct)} distinct seeded blocks cycled",
                    "l2": "per-block inputs (63 MB) live in HBM; no flush", "parallelism": f"independent replica per GPU x{world}"},
-        "latency_us": {"p50": p50, "p99": p99, "min": float(lat.min()), "max": float(lat.max())},
+        "latency_us": {"p50": p50, "p99": p99, "min": float(lat.min()), "max": float(lat.max()),
+                       "host_enqueue_per_block": host_us, "graph_replay_per_block": graph_us,
+                       "graph_error": graph_err},
         "roofline": {"bound": "hbm", "kernel": "block_step (3 launches)", "achieved": alg / (p50 * 1e-6) / 1e9,
                      "peak": peak, "unit": "GB/s", "frac": alg / (p50 * 1e-6) / 1e9 / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": None, "algorithmic_bytes_per_launch": alg},
@@ -516,6 +595,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=None,
                     help="oracle rows per reference-arm step (default: sized so the whole run stays near a minute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=7, help="head chunks pipelined through the e2e step")
     args = ap.parse_args()
     w = workloads.CONFIGS[args.config]
     if args.impl == "reference":

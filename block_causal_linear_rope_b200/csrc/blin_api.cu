@@ -50,6 +50,19 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------------- geometry
+// SMs of the current device (cached per device).
+static int device_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 struct Plan {
     KGeom g;
     int d;
@@ -106,7 +119,17 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
     const long long max_blk_tok = (long long)(one_block ? T : (F < T ? F : T)) * g.HW;
     g.cpb = (int)((max_blk_tok + kChunk - 1) / kChunk);
     if (g.cpb < 1) g.cpb = 1;
-    const int qtok = kQTiles * kTile;
+    // Output groups of up to kQTiles query tiles; a call with few tiles (a decode
+    // block) uses smaller groups, so that every pipeline of the output kernel gets
+    // several (results do not depend on the grouping).
+    g.qgt = kQTiles;
+    if (!for_size) {
+        const long long tiles_per_blk = (max_blk_tok + kTile - 1) / kTile;
+        const long long pipelines = 2LL * device_sms();
+        while (g.qgt > 2 && (long long)g.BH * g.nblk * ((tiles_per_blk + g.qgt - 1) / g.qgt) < 4 * pipelines)
+            g.qgt /= 2;
+    }
+    const int qtok = g.qgt * kTile;
     g.qcpb = (int)((max_blk_tok + qtok - 1) / qtok);
     if (g.qcpb < 1) g.qcpb = 1;
     g.pt = split[0] / 2;

@@ -13,7 +13,7 @@ namespace blin {
 constexpr int kTile = 128;
 constexpr int kChunkTiles = 8;
 constexpr int kChunk = kTile * kChunkTiles;  // 1024 tokens: fixed per block => bit-exact streaming
-constexpr int kQTiles = 8;                    // output tiles per CTA
+constexpr int kQTiles = 8;                    // most query tiles per output group
 
 // Geometry of one call, shared by all kernels of that call.
 struct KGeom {
@@ -25,7 +25,8 @@ struct KGeom {
     int first_end;        // relative frame at which block 0 ends
     int nblk;             // blocks touched by the call
     int cpb;              // state chunks per block (stride of the partial buffer)
-    int qcpb;             // output CTAs per block (grid.x of the output kernel)
+    int qcpb;             // output groups per block
+    int qgt;              // query tiles per output group (<= kQTiles; fewer when a call has few tiles)
     int pt, py, px;       // RoPE pairs per axis (t, y, x)
     float eps;
     const float2 *tab;    // (cos, sin): [T][pt] then [Hg][py] then [Wg][px]

@@ -644,7 +644,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
     using C = P2<D>;
     constexpr int NP = C::NP, NL = C::NL, NO = C::NO, NA = C::NACC, NT = C::NT, TB = C::TB, ROWB = C::ROWB;
     constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, C::N, 0, 0);
-    constexpr int QG = kQTiles * kTile;  // tokens per group
+    const int QG = g.qgt * kTile;  // tokens per group
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
