@@ -9,7 +9,7 @@
 
 namespace blin {
 
-// Tokens per TMA tile / MMA row block, tiles per state chunk and per output CTA.
+// Tokens per TMA tile (and MMA row block) and tiles per state chunk.
 constexpr int kTile = 128;
 constexpr int kChunkTiles = 8;
 constexpr int kChunk = kTile * kChunkTiles;  // 1024 tokens: fixed per block => bit-exact streaming

@@ -227,12 +227,10 @@ __device__ __forceinline__ uint4 b_operand_chunk(const float *pre, int item) {
 // ============================================================================ shared control
 __device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
 
-// Tiles of a work unit alternate between two transform groups (tile k goes to
-// group k & 1).  A group's first tile of a unit is tile 0 or 1; it then steps
-// by two tiles.  The producer ends the stream with two markers: -1 (passed on
-// through the operand ring) for the group that sees the end first, -2 for the
-// other group, which just stops.
-constexpr int kEndFirst = -1, kEndSecond = -2;
+// Each pipeline's producer ends its tile stream with this unit id in the
+// landing-slot record; the transform warps pass it on to the MMA issuer through
+// the operand ring, and both stop there.
+constexpr int kEndFirst = -1;
 
 // One mbarrier arrival for the whole warp, after every lane's shared-memory
 // accesses (and tcgen05 loads, fenced by the caller) are ordered before it.
