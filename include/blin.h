@@ -125,11 +125,14 @@ BLIN_API blin_status blin_state_reserve(blin_state *st, long max_block_tokens, b
 
 /* ---------------------------------------------------------------- prefill */
 
-/* Workspace bytes blin_prefill needs for this shape (0 on invalid input). */
+/* Workspace bytes blin_prefill needs for this shape (0 on invalid input).  A
+ * call uses its workspace until its last kernel has finished: calls that may
+ * run at the same time (on different streams) need separate workspaces. */
 BLIN_API size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom *g);
 
 /* Block-causal linear attention over a whole latent video (or a continuation).
- *   q, k, v  device [B][H][N][d] of dtype dt;  o  device [B][H][N][d] output
+ *   q, k, v  device [B][H][N][d] of dtype dt;  o  device [B][H][N][d] output,
+ *            which must not overlap q, k or v
  *   st       optional cache.  NULL: start from S = 0, z = 0, t0 = 0.
  *            Otherwise start from its (S, z) with t0 = its t_next, and on
  *            return (in stream order) it holds the final (S, z) with
