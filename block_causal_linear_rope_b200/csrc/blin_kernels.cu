@@ -148,12 +148,9 @@ static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, i
 
 cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
                         float *z_out, cudaStream_t s) {
-    const long long cols = (long long)g.BH * ((d * d + d) / 4);  // (head, float4 column) pairs
-    const dim3 grid((unsigned)((cols + kScanSlice - 1) / kScanSlice));
-    const int groups = g.nblk < 32 ? (g.nblk > 0 ? g.nblk : 1) : 32;  // thread groups of 32 columns
-    const int seg = g.nblk < kScanSeg ? (g.nblk > 0 ? g.nblk : 1) : kScanSeg;
-    const int smem = seg * kScanSlice * (int)sizeof(float4);
-    cudaError_t e = launch_pdl(scan_kernel, grid, dim3(kScanSlice * groups), smem, s, g, d, S_in, z_in, S_out, z_out);
+    const long long cols = (long long)g.BH * ((d * d + d) / 4);  // (head, float4 column) pairs: one thread each
+    const dim3 grid((unsigned)((cols + 255) / 256));
+    cudaError_t e = launch_pdl(scan_kernel, grid, dim3(256), 0, s, g, d, S_in, z_in, S_out, z_out);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -53,69 +53,64 @@ __global__ void rope_table_kernel(float2 *tab, int T, int t0, int Hg, int Wg, in
 // The order depends only on the block's own length, so a block-by-block
 // stream reproduces a one-shot prefill bit for bit.  (Talk transcript: the
 // new state is the cached state plus the block's contribution.)
-// One CTA per (head, 32 float4 columns): thread groups form the block sums
-// P_b in parallel (their chunk loads all in flight), then one group runs the
-// chain over blocks from shared memory.  Blocks are taken kScanSeg at a time.
-constexpr int kScanSlice = 32;  // (head, float4 column) pairs per CTA: one per lane
-constexpr int kScanBatch = 8;   // chunk loads issued together per block
-constexpr int kScanSeg = 64;    // blocks staged in shared memory at once (at most 32 KB)
+// One thread per (head, float4 column), all heads' columns laid end to end, so
+// the launch is one wave whatever the block count.
+constexpr int kScanLoads = 16;  // chunk partial loads in flight per thread
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
-// Inclusive scan over blocks of the chunk partial states, per head, in a fixed
-// order: S_<=b = S_<=b-1 + ((c0 + c1) + c2 ...) over block b's chunks, starting
-// from the carried state (S_in, z_in) or zero.  The (head, float4 column)
-// pairs of all heads are laid end to end and each CTA takes 32 consecutive
-// ones, so no lane idles on a head's ragged last columns; thread group j of a
-// CTA sums the chunks of blocks j, j + groups, ... into shared memory and group
-// 0 then chains them.
-__global__ void __launch_bounds__(1024) scan_kernel(KGeom g, int d, const float *S_in, const float *z_in,
-                                                    float *S_out, float *z_out) {
-    extern __shared__ float4 sm[];  // [min(nblk, kScanSeg)][kScanSlice]
+// Each thread walks its column's (block, chunk) sequence in order, keeping
+// kScanLoads loads in flight across block boundaries; consecutive threads read
+// consecutive columns.
+__global__ void __launch_bounds__(256) scan_kernel(KGeom g, int d, const float *S_in, const float *z_in,
+                                                   float *S_out, float *z_out) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");  // chunk partials come from the previous kernel
     const int E4 = (d * d + d) / 4;
-    const int col = threadIdx.x % kScanSlice, grp = threadIdx.x / kScanSlice;
-    const int ngrp = blockDim.x / kScanSlice;
-    const long long f = (long long)blockIdx.x * kScanSlice + col;
-    const bool live = f < (long long)g.BH * E4;
-    const int bh = live ? (int)(f / E4) : 0, e4 = live ? (int)(f - (long long)bh * E4) : 0;
-    const float4 *part = reinterpret_cast<const float4 *>(g.part);
-    float4 *prefix = reinterpret_cast<float4 *>(g.prefix);
+    const long long f = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (f >= (long long)g.BH * E4) return;
+    const int bh = (int)(f / E4), e4 = (int)(f - (long long)bh * E4);
+    const float4 *part = reinterpret_cast<const float4 *>(g.part) + (size_t)bh * g.nblk * g.cpb * E4 + e4;
+    float4 *prefix = reinterpret_cast<float4 *>(g.prefix) + (size_t)bh * g.nblk * E4 + e4;
+    auto nchunks = [&](int b) {
+        return ((block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
+    };
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (grp == 0 && live && S_in != nullptr)
+    if (S_in != nullptr)
         acc = 4 * e4 < d * d ? reinterpret_cast<const float4 *>(S_in + (size_t)bh * d * d)[e4]
                              : reinterpret_cast<const float4 *>(z_in + (size_t)bh * d)[e4 - d * d / 4];
-    for (int b0 = 0; b0 < g.nblk; b0 += kScanSeg) {
-        const int nb = min(kScanSeg, g.nblk - b0);
-        for (int bl = grp; bl < nb; bl += ngrp) {
-            if (!live) continue;
-            const int b = b0 + bl;
-            const int n = ((block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
-            const float4 *p = part + ((size_t)(bh * g.nblk + b) * g.cpb) * E4 + e4;
-            float4 v[kScanBatch];
+    // issue cursor (ib, ic) and consume cursor (cb, cc) over the (block, chunk) sequence
+    int ib = 0, ic = 0, in = g.nblk > 0 ? nchunks(0) : 0;
+    int cb = 0, cc = 0, cn = in;
+    float4 pb = make_float4(0.f, 0.f, 0.f, 0.f);
+    while (cb < g.nblk) {
+        float4 v[kScanLoads];
 #pragma unroll
-            for (int c = 0; c < kScanBatch; ++c)
-                if (c < n) v[c] = __ldcg(p + (size_t)c * E4);
-            float4 pb = v[0];
-#pragma unroll
-            for (int c = 1; c < kScanBatch; ++c)
-                if (c < n) pb = f4add(pb, v[c]);
-            for (int c = kScanBatch; c < n; ++c) pb = f4add(pb, __ldcg(p + (size_t)c * E4));
-            sm[bl * kScanSlice + col] = pb;
-        }
-        __syncthreads();
-        if (grp == 0 && live) {
-            for (int bl = 0; bl < nb; ++bl) {
-                acc = f4add(acc, sm[bl * kScanSlice + col]);
-                prefix[((size_t)bh * g.nblk + b0 + bl) * E4 + e4] = acc;
+        for (int j = 0; j < kScanLoads; ++j) {
+            if (ib < g.nblk) {
+                v[j] = __ldcg(part + ((size_t)ib * g.cpb + ic) * E4);
+                if (++ic == in) {
+                    ic = 0;
+                    if (++ib < g.nblk) in = nchunks(ib);
+                }
             }
         }
-        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kScanLoads; ++j) {
+            if (cb < g.nblk) {
+                pb = cc == 0 ? v[j] : f4add(pb, v[j]);
+                if (++cc == cn) {  // block cb complete
+                    acc = f4add(acc, pb);
+                    prefix[(size_t)cb * E4] = acc;
+                    cc = 0;
+                    if (++cb < g.nblk) cn = nchunks(cb);
+                }
+            }
+        }
     }
-    if (grp == 0 && live && S_out != nullptr) {
+    if (S_out != nullptr) {
         if (4 * e4 < d * d)
             reinterpret_cast<float4 *>(S_out + (size_t)bh * d * d)[e4] = acc;
         else
