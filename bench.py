@@ -220,6 +220,16 @@ def oracle_sample(w: workloads.Workload, q, k, v, rows_total: int, seed: int = 0
     return rows_total * qs.shape[0] / dt, dt
 
 
+def oracle_recurrence_rate(w: workloads.Workload, q, k, v):
+    """Time the float64 state-form oracle (O(N d^2)) on the whole workload: token*heads per second."""
+    import oracle
+    pos, blk = oracle.grid(w.T, w.Hg, w.Wg, w.F)
+    t0 = time.perf_counter()
+    oracle.recurrence(q, k, v, pos, blk, w.split, w.theta, w.eps)
+    dt = time.perf_counter() - t0
+    return w.B * w.H * w.N / dt, dt
+
+
 def omp_threads() -> int:
     n = os.environ.get("OMP_NUM_THREADS")
     return int(n) if n else (os.cpu_count() or 1)
@@ -442,9 +452,13 @@ def run_blin(args, w):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, secs = oracle_sample(w, q, k, v, args.cpu_rows)
+        rec_rate, rec_secs = oracle_recurrence_rate(w, q, k, v)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
                                 "sample": f"{args.cpu_rows} seeded query rows x {w.B * w.H} heads of {w.name}, "
-                                          f"explicit O(N^2) float64 pair sum, {secs:.1f} s"}
+                                          f"explicit O(N^2) float64 pair sum, {secs:.1f} s",
+                                "recurrence": {"value": rec_rate, "unit": UNIT,
+                                               "sample": f"the whole {w.name} workload through the float64 "
+                                                         f"state-form oracle (O(N d^2)), {rec_secs:.1f} s"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
