@@ -260,7 +260,7 @@ struct P1 {
     static constexpr int RINGS = NP * (2 * NO + NK + NV) * TB;  // operand, K and V rings of all pipelines
     static constexpr int FIXED = RINGS + TB + CTRL + 1024;  // + RoPE table
     static constexpr int THREADS = 32 * 6 * NP;  // warps [0, 4NP) transform, then NP producers, NP MMA issuers
-    static_assert(NP * NBAR * 8 <= BARS, "mbarriers overflow their area");
+    static_assert(NP * (NBAR + 1) * 8 <= BARS, "mbarriers (+ one drain barrier per pipeline) overflow their area");
     static_assert(BARS + 4 * NP * (4 * NK + 4 * NO) + 16 <= CTRL, "control block overflow");
     static_assert(NV > NO, "an operand slot's release is read from the V ring's tile-done barriers");
     // the B operand's second N atom (the ones block) sits above every V slot
@@ -330,6 +330,8 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
     auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NK + NV + s); };
     auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NK + NV + NO + a); };
     auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NK + NV + NO + NA + a); };
+    // drain: one final commit, so that the MMA thread leaves only after all its MMAs are done
+    const uint32_t drain = ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + pipe);
 
     const int units = g.cpb * g.nblk * g.BH;
     const int per_c = g.nblk * g.BH;
@@ -354,6 +356,7 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                 ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + NO + a), 1);       // accf: commit
                 ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + NO + NA + a), 4);  // acce: transform warps
             }
+            ptx::mbar_init(ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + p), 1);  // drain
         }
         flags[0] = 0;
         ptx::fence_mbar_init();
@@ -459,6 +462,10 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                     ++nu;
                 }
             }
+            // every MMA (and the arrivals of the commits above) completes before the CTA's
+            // final barrier and TMEM release, also when a wait gave up
+            ptx::mma_commit(drain);
+            if (!ptx::mbar_wait_bounded(drain, 0, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) flags[0] = 1;
         }
     } else {
         // ------------------------------------------------------------ transform warps: one row per thread
@@ -615,7 +622,7 @@ struct P2 {
     static constexpr int PIPE = (NL * TB + NO * 2 * TB + TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
     static constexpr int FIXED = NP * PIPE + CTRL + 1024;  // + RoPE table
     static constexpr int THREADS = 32 * 10 * NP;  // per pipeline: 4 transform, 4 epilogue, producer, MMA warps
-    static_assert(NP * NBAR * 8 <= BARS, "mbarriers overflow their area");
+    static_assert(NP * (NBAR + 1) * 8 <= BARS, "mbarriers (+ one drain barrier per pipeline) overflow their area");
     static_assert(BARS + 16 + NP * 4 * 8 * (NL + NO) <= CTRL, "control block overflow");
     static_assert(TCOLS <= 512, "TMEM holds 512 columns");
     static_assert(PIPE % 1024 == 0, "pipelines keep 1024-byte alignment");
@@ -674,6 +681,8 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
     auto pfull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + s); };
     auto pempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + 2 + s); };
     auto bempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + 4 + s); };
+    // drain: one final commit, so that the MMA thread leaves only after all its MMAs are done
+    const uint32_t drain = ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + pipe);
 
     const int units = g.qcpb * g.nblk * g.BH;
     const int per_q = g.nblk * g.BH;
@@ -699,6 +708,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
                 ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + 2 + s), 4);  // pempty: transform warps
                 ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + 4 + s), 1);  // bempty: commit
             }
+            ptx::mbar_init(ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + p), 1);  // drain
         }
         flags[0] = 0;
         ptx::fence_mbar_init();
@@ -807,6 +817,10 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
                 ptx::mma_commit(tdone(k % NT));
                 if (last) ptx::mma_commit(bempty(ord & 1));
             }
+            // every MMA (and the arrivals of the commits above) completes before the CTA's
+            // final barrier and TMEM release, also when a wait gave up
+            ptx::mma_commit(drain);
+            if (!ptx::mbar_wait_bounded(drain, 0, watchdog, WD_OUT_MMA, kWaitLimitNs)) flags[0] = 1;
         }
     } else if (warp < 4 * NP) {
         // ------------------------------------------------------------ transform warps: one row per thread
