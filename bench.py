@@ -1,14 +1,21 @@
 """Throughput of block-causal linear attention (prefill) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl blin|reference] [--config 480p]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl blin|reference]
+                    [--config 480p|720p|wide|decode]
 
-One step = one blin_prefill of the whole workload (RoPE table, partial states,
-block scan, output) on inputs already resident in HBM.  The workload defaults
-to the 480p-like latent video: B=1, H=70, d=32, 21 x 30 x 52 tokens, blocks of
-3 frames, bf16 storage.  Inputs (587 MB moved per step) are larger than L2, so
-no flush is needed between steps.  With N > 1 GPUs every rank runs its own
-independent copy of the workload (weak scaling; heads/videos never exchange
-data) and the step time is the max over ranks.
+One step = one blin_prefill of the whole workload (on the tensor-core path three
+kernels: partial states, block scan, output) on inputs already resident in HBM.
+The workload defaults to the 480p-like latent video: B=1, H=70, d=32,
+21 x 30 x 52 tokens, blocks of 3 frames, bf16 storage.  Inputs (587 MB moved
+per step) are larger than L2, so no flush is needed between steps.  The line
+also reports the per-kernel roofline, an end-to-end figure with host copies,
+the float64 oracle's CPU rate and the SM clocks seen while timing.  With N > 1
+GPUs every rank runs its own independent copy of the workload (weak scaling;
+heads/videos never exchange data) and the step time is the max over ranks.
+
+``--config decode`` times 80 blin_block_step calls (one 3-frame block each)
+instead: per-block latency percentiles, the same calls replayed as a CUDA
+graph, and whether device memory stays flat.
 
 ``--impl reference`` times the float64 CPU oracle (the only reference this
 method has) on a bounded sample of the same workload and prints the same line
