@@ -1,25 +1,29 @@
-"""Throughput of block-causal linear attention (prefill) on B200.
+"""Throughput of block-causal linear attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl blin|reference]
-                    [--config 480p|720p|wide|decode]
+                    [--config all|720p|480p|wide|decode|denoise]
 
-One step = one blin_prefill of the whole workload (on the tensor-core path three
-kernels: partial states, block scan, output) on inputs already resident in HBM.
-The workload defaults to the 480p-like latent video: B=1, H=70, d=32,
-21 x 30 x 52 tokens, blocks of 3 frames, bf16 storage.  Inputs (587 MB moved
-per step) are larger than L2, so no flush is needed between steps.  The line
-also reports the per-kernel roofline, an end-to-end figure with host copies,
-the float64 oracle's CPU rate and the SM clocks seen while timing.  With N > 1
-GPUs every rank runs its own independent copy of the workload (weak scaling;
-heads/videos never exchange data) and the step time is the max over ranks.
+Headline (default ``--config all``): one step = one blin_prefill of the
+720p-like latent video (B=1, H=70, d=32, 21 x 45 x 80 tokens, blocks of 3
+frames, bf16 storage, lognormal Q/K channel scales) on inputs already resident
+in HBM.  The inputs (1355 MB moved per step) are larger than L2, so no flush is
+needed between steps.  The line also reports the per-kernel roofline, an
+end-to-end figure with host copies inside the timed region, the float64
+oracle's CPU rate and the SM clocks seen while timing, plus sub-records:
 
-``--config decode`` times 80 blin_block_step calls (one 3-frame block each)
-instead: per-block latency percentiles, the same calls replayed as a CUDA
-graph, and whether device memory stays flat.
+  480p, wide   the same prefill measurement on the 480p-like and the
+               wide-head (B=4, H=32, d=64, one-frame blocks) workloads;
+  decode       80 blin_block_step calls (one 3-frame 30 x 52 block each,
+               commit=1): per-block latency percentiles, the same calls
+               replayed as one CUDA graph, device memory after every block;
+  denoise      16 blocks, each denoised by 4 read-only block steps (fresh
+               Q/K/V, commit=0) and then committed once, replayed as a graph.
 
-``--impl reference`` times the float64 CPU oracle (the only reference this
-method has) on a bounded sample of the same workload and prints the same line
-with ``"impl": "reference"``.
+With N > 1 GPUs every rank runs its own independent copy of the workload (weak
+scaling; heads and videos never exchange data) and each time is the max over
+ranks.  ``--impl reference`` times the float64 CPU oracle (the only reference
+this method has) on a bounded sample of the same workload and prints the same
+line with ``"impl": "reference"``.
 """
 from __future__ import annotations
 
@@ -281,30 +285,37 @@ def config_dict(w, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_blin(args, w):
+def _load_blin(args):
     import torch
 
     world, rank, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     import block_causal_linear_rope_b200 as blin
+    return torch, blin, world, rank, local
 
+
+def _prefill_args(blin, w, qd, kd, vd, od, ws, stream_ptr):
+    """Pre-marshalled C-ABI arguments of one blin_prefill call (no state)."""
+    geom = blin._geom(w.T, w.Hg, w.Wg, w.F, w.split, w.theta, w.eps)
+    return (ctypes.c_void_p(qd.data_ptr()), ctypes.c_void_p(kd.data_ptr()), ctypes.c_void_p(vd.data_ptr()),
+            ctypes.c_void_p(od.data_ptr()), blin.BF16 if w.dtype == "bf16" else blin.F32, w.B, w.H, w.d,
+            ctypes.byref(geom), None, ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(stream_ptr)), geom
+
+
+def measure_prefill(args, w, torch, blin, world, rank, clk, full: bool):
+    """Device-resident prefill steps of workload w: the headline numbers, per-kernel event times and
+    the roofline; with `full`, also the end-to-end figure (host copies inside the timed region) and
+    the CPU baseline.  Returns the record (a dict)."""
     dt_t = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     wr = replica_workload(w, rank)
     q, k, v = workloads.call_tensors(wr)
     qh, kh, vh = (torch.from_numpy(x).to(dt_t).pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.to("cuda") for x in (qh, kh, vh))
     od = torch.empty_like(qd)
-    oh = torch.empty_like(qh).pin_memory()
     grid = (w.T, w.Hg, w.Wg)
     ws = torch.empty(blin.workspace_size(w.B, w.H, w.d, grid, w.F, w.split, w.theta, w.eps),
                      dtype=torch.uint8, device="cuda")
-
-    # pre-marshalled C-ABI arguments: the timed loop calls blin_prefill directly
-    geom = blin._geom(w.T, w.Hg, w.Wg, w.F, w.split, w.theta, w.eps)
-    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    cargs = (ctypes.c_void_p(qd.data_ptr()), ctypes.c_void_p(kd.data_ptr()), ctypes.c_void_p(vd.data_ptr()),
-             ctypes.c_void_p(od.data_ptr()), blin.BF16 if w.dtype == "bf16" else blin.F32, w.B, w.H, w.d,
-             ctypes.byref(geom), None, ctypes.c_void_p(ws.data_ptr()), ws.numel(), stream)
+    cargs, geom = _prefill_args(blin, w, qd, kd, vd, od, ws, torch.cuda.current_stream().cuda_stream)
     prefill_c = blin.lib.blin_prefill
 
     def step():
@@ -315,55 +326,73 @@ def run_blin(args, w):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    path = blin.last_path()
     barrier(world)
     torch.cuda.synchronize()
-
     timer = blin.LaunchTimer()
     sets = [timer.new_set() for _ in range(args.steps)]
     arm = blin.LaunchTimer.arm_set
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        time.sleep(0.25)  # let the sampler start
-        # (1) the headline: K steps back to back, timed by two events on the
-        # launching stream; nothing is recorded between the kernels
-        n0 = blin.launch_count()
-        t_wall = time.time()
-        start.record()
-        for _ in range(args.steps):
-            step()
-        end.record()
-        torch.cuda.synchronize()
-        clk.timed(t_wall, time.time())
-        launches = blin.launch_count() - n0
-        barrier(world)
-        torch.cuda.synchronize()
-        # (2) the same K steps again with an event pair around every launch, for
-        # the per-kernel durations behind the roofline (events between kernels
-        # also stop the next kernel from starting early, so this pass is slower)
-        t_wall = time.time()
-        for i in range(args.steps):
-            arm(sets[i])
-            step()
-        torch.cuda.synchronize()
-        clk.timed(t_wall, time.time())
-        blin.lib.blin_set_timing_events(None, 0)
-        time.sleep(0.25)
+    # (1) the headline: K steps back to back, timed by two events on the launching stream;
+    # nothing is recorded between the kernels
+    n0 = blin.launch_count()
+    t_wall = time.time()
+    start.record()
+    for _ in range(args.steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    clk.timed(t_wall, time.time())
+    launches = blin.launch_count() - n0
     barrier(world)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / args.steps
-    ms = max_over_ranks(ms, world)
+    # (2) the same K steps again with an event pair around every launch, for the per-kernel
+    # durations behind the roofline (events between kernels also keep the next kernel from
+    # starting early, so this pass is slower)
+    t_wall = time.time()
+    for i in range(args.steps):
+        arm(sets[i])
+        step()
+    torch.cuda.synchronize()
+    clk.timed(t_wall, time.time())
+    blin.lib.blin_set_timing_events(None, 0)
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, world)
     per_kernel = timer.elapsed_ms()
     avg = {kname: sum(d[kname] for d in per_kernel) / len(per_kernel) for kname in blin.KERNELS}
-    # the tensor-core path builds its RoPE tables inside the kernels: 3 launches a step
-    table_launched = launches != 3 * args.steps
     status = blin.device_status()
     if status != 0:
         raise SystemExit(f"kernel watchdog fired (code {status})")
+
+    units = w.B * w.H * w.N  # token*heads per GPU per step
+    elem = 2 if w.dtype == "bf16" else 4
+    launched = {kname: avg[kname] for kname in blin.KERNELS if blin.KERNEL_BYTES_PER_UNIT.get(kname) is not None
+                and avg[kname] > 0.0005}
+    alg = {kname: blin.KERNEL_BYTES_PER_UNIT[kname] * w.d * elem * units for kname in launched}
+    dom = max(launched, key=lambda k_: launched[k_])
+    peak, peak_kind = hbm_peak()
+    achieved = alg[dom] / (launched[dom] * 1e-3) / 1e9
+    whole = 4 * units * w.d * elem / (ms * 1e-3) / 1e9
+    rec = {
+        "value": job_throughput(units, world, ms), "unit": UNIT, "ms_per_step": ms, "path": path,
+        "workload": config_dict(w, world)["workload"],
+        "hbm_gbs_whole_step": whole, "hbm_frac_whole_step": whole / peak,
+        "kernel_ms": launched,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": recorded_traffic(dom, w.name),
+                     "algorithmic_bytes_per_launch": alg[dom]},
+        "gpu_launches": launches,
+    }
+    if not full:
+        return rec
 
     # ---- end to end through the C ABI: pinned host inputs in, host output back.  Heads are
     # independent and contiguous ([B*H][N][d]), so the step is cut into head chunks that flow
     # through three streams (copy in, compute, copy out): one blin_prefill per chunk, and the
     # host-to-device and device-to-host copies overlap each other and the kernels.
+    oh = torch.empty_like(qh).pin_memory()
     h2d = 3 * qh.numel() * qh.element_size()
     d2h = oh.numel() * oh.element_size()
     od_ref = od.clone()  # the device-resident steps' output
@@ -427,91 +456,64 @@ def run_blin(args, w):
     # the chunked output must equal the one-call output (same kernels, same inputs, heads independent)
     if not torch.equal(oh.to("cuda"), od_ref):
         raise SystemExit("end-to-end output differs from the device-resident step")
-
-    units = w.B * w.H * w.N  # token*heads per GPU per step
-    value = job_throughput(units, world, ms)
-    e2e_value = job_throughput(units, world, e_ms)
-
-    # ---- roofline of the dominant kernel (algorithmic bytes / live event time)
-    elem = 2 if w.dtype == "bf16" else 4
-    alg = {"partial_states": 2 * units * w.d * elem,  # K and V read
-           "output": 2 * units * w.d * elem}          # Q read, O written
-    dom = max(("partial_states", "output"), key=lambda k_: avg[k_])
-    peak, peak_kind = hbm_peak()
-    achieved = alg[dom] / (avg[dom] * 1e-3) / 1e9
-    whole = 4 * units * w.d * elem / (ms * 1e-3) / 1e9
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": config_dict(w, world),
-        "hbm_gbs_whole_step": whole, "hbm_frac_whole_step": whole / peak,
-        "kernel_ms": {kname: avg[kname] for kname in blin.KERNELS if table_launched or kname != "rope_table"},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
-                     "traffic": recorded_traffic(dom, w.name),
-                     "algorithmic_bytes_per_launch": alg[dom]},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e_ms, "head_chunks": nchunk},
-        "gpu_launches": launches,
-        "clocks": clk.summary(),
-    }
+    rec["e2e"] = {"value": job_throughput(units, world, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "head_chunks": nchunk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, secs = oracle_sample(w, q, k, v, args.cpu_rows)
+        # a bounded sample of about 10-20 s: rows scaled by the keys each row sees
+        cpu_rows = args.cpu_rows or max(64, int(2000 * 32760 / w.N))
+        rate, secs = oracle_sample(w, q, k, v, cpu_rows)
         rec_rate, rec_secs = oracle_recurrence_rate(w, q, k, v)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
-                                "sample": f"{args.cpu_rows} seeded query rows x {w.B * w.H} heads of {w.name}, "
-                                          f"explicit O(N^2) float64 pair sum, {secs:.1f} s",
-                                "recurrence": {"value": rec_rate, "unit": UNIT,
-                                               "sample": f"the whole {w.name} workload through the float64 "
-                                                         f"state-form oracle (O(N d^2)), {rec_secs:.1f} s"}}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+        rec["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+                               "sample": f"{cpu_rows} seeded query rows x {w.B * w.H} heads of {w.name}, "
+                                         f"explicit O(N^2) float64 pair sum, {secs:.1f} s",
+                               "recurrence": {"value": rec_rate, "unit": UNIT,
+                                              "sample": f"the whole {w.name} workload through the float64 "
+                                                        f"state-form oracle (O(N d^2)), {rec_secs:.1f} s"}}
+    return rec
 
 
-# ----------------------------------------------------------------------------- decode (block_step) latency
-def run_decode(args, w):
-    """Minute-long autoregressive decode: w.steps calls of blin_block_step (one block of w.F frames
-    each, commit=1) against the constant-size (S, z) cache; per-block latency and device memory."""
-    import torch
-
-    world, rank, local = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    import block_causal_linear_rope_b200 as blin
-
+def measure_decode(args, w, torch, blin, world, rank, clk, denoise_steps: int = 0):
+    """Minute-long autoregressive decode: w.steps blin_block_step calls (one block of w.F frames each)
+    against the constant-size (S, z) cache.  With denoise_steps = K > 0, every block is first run K
+    times read-only (commit=0, fresh Q/K/V each: denoising steps) and then committed once.
+    Per-block latency from events around each block, the same sequence replayed as one CUDA graph,
+    device memory after every block, and the state's size."""
     wr = replica_workload(w, rank)
     dt_t = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     nb, F = w.steps, w.F
-    # inputs resident on the device before timing: 8 distinct seeded blocks, cycled over the
-    # nb calls (drawing all 80 blocks' 2.5e9 normals would take the host about a minute)
-    distinct = [tuple(torch.from_numpy(workloads.block_tensor(wr, tid, b, F)).to("cuda", dt_t) for tid in (0, 1, 2))
-                for b in range(min(nb, 8))]
-    blocks = [distinct[b % len(distinct)] for b in range(nb)]
-    out = torch.empty_like(blocks[0][0])
+    calls_per_block = denoise_steps + 1
+    # inputs resident on the device before timing: a few distinct seeded blocks, cycled over the
+    # calls (drawing all 80 blocks' 2.5e9 normals would take the host about a minute)
+    ndist = min(nb * calls_per_block, 8)
+    distinct = [tuple(torch.from_numpy(workloads.block_tensor(wr.with_(seed=wr.seed + 1000 * j), tid, 0, F))
+                      .to("cuda", dt_t) for tid in (0, 1, 2)) for j in range(ndist)]
+    out = torch.empty_like(distinct[0][0])
     st = blin.BlockState(w.B, w.H, w.d)
     st.reserve(F * w.HW)
-    split = (ctypes.c_int * 3)(*w.split)
+    geom = blin._geom(F, w.Hg, w.Wg, F, w.split, w.theta, w.eps)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     dt_c = blin.BF16 if w.dtype == "bf16" else blin.F32
     step_c = blin.lib.blin_block_step
-    cargs = [(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
-              ctypes.c_void_p(out.data_ptr()), dt_c, w.B, w.H, w.d, w.Hg, w.Wg, F, ctypes.byref(split), w.theta,
-              w.eps, st.handle, 1, stream) for (q, k, v) in blocks]
+    cargs = []
+    for b in range(nb):
+        for s_ in range(calls_per_block):
+            q, k, v = distinct[(b * calls_per_block + s_) % ndist]
+            commit = 1 if s_ == denoise_steps else 0
+            cargs.append((ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+                          ctypes.c_void_p(out.data_ptr()), dt_c, w.B, w.H, w.d, ctypes.byref(geom), st.handle,
+                          commit, stream))
 
     def sequence(events=None):
         st.reset()
-        for i, a in enumerate(cargs):
+        for b in range(nb):
             if events is not None:
-                events[i][0].record()
-            rc = step_c(*a)
-            if rc != 0:
-                raise RuntimeError(blin.lib.blin_last_error().decode())
+                events[b][0].record()
+            for a in cargs[b * calls_per_block:(b + 1) * calls_per_block]:
+                rc = step_c(*a)
+                if rc != 0:
+                    raise RuntimeError(blin.lib.blin_last_error().decode())
             if events is not None:
-                events[i][1].record()
+                events[b][1].record()
 
     for _ in range(max(1, args.warmup // 5)):
         sequence()
@@ -521,29 +523,21 @@ def run_decode(args, w):
     lat, mem_flat = [], True
     reps = max(1, min(args.steps // 100, 10))
     barrier(world)
-    with ClockSampler(local) as clk:
-        time.sleep(0.25)
-        t_wall = time.time()
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        start.record()
-        for _ in range(reps):
-            sequence(evs)
-            torch.cuda.synchronize()
-            lat += [a.elapsed_time(b) * 1e3 for a, b in evs]
-            mem_flat &= torch.cuda.mem_get_info()[0] == free0
-        end.record()
+    t_wall = time.time()
+    for _ in range(reps):
+        sequence(evs)
         torch.cuda.synchronize()
-        clk.timed(t_wall, time.time())
-        time.sleep(0.25)
-    # host time to enqueue one block (plan, tensor maps, launches): with the GPU this fast, the
-    # stream-launched latency above is set by it
+        lat += [a.elapsed_time(b) * 1e3 for a, b in evs]
+        mem_flat &= torch.cuda.mem_get_info()[0] == free0
+    clk.timed(t_wall, time.time())
+    # host time to enqueue one block (plan, tensor maps, launches)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     sequence()
     host_us = (time.perf_counter() - t0) / nb * 1e6
     torch.cuda.synchronize()
-    # the same nb calls captured once in a CUDA graph and replayed: per-block device time
-    # without host launch overhead
+    # the same calls captured once in a CUDA graph and replayed: per-block device time without
+    # host launch overhead
     graph_us, graph_err = None, None
     try:
         cg = torch.cuda.CUDAGraph()
@@ -564,7 +558,7 @@ def run_decode(args, w):
             cg.replay()
         g1.record()
         torch.cuda.synchronize()
-        graph_us = g0.elapsed_time(g1) * 1e3 / (reps * nb)
+        graph_us = max_over_ranks(g0.elapsed_time(g1) * 1e3 / (reps * nb), world)
         del cg
     except Exception as exc:  # capture unsupported: report why, keep the stream numbers
         graph_err = str(exc).splitlines()[0][:200]
@@ -573,33 +567,74 @@ def run_decode(args, w):
         raise SystemExit(f"kernel watchdog fired (code {status})")
     lat = np.array(lat)
     units = w.B * w.H * F * w.HW
-    p50 = float(np.percentile(lat, 50))
-    p99 = float(np.percentile(lat, 99))
-    p50 = max_over_ranks(p50, world)
+    p50 = max_over_ranks(float(np.percentile(lat, 50)), world)
+    p99 = max_over_ranks(float(np.percentile(lat, 99)), world)
     elem = 2 if w.dtype == "bf16" else 4
-    alg = 4 * units * w.d * elem + 2 * st.nbytes  # Q, K, V read, O written; state read and written
+    # per call: Q, K, V read, O written; state read (and written by the commit)
+    alg_call = 4 * units * w.d * elem + st.nbytes
+    alg_block = calls_per_block * alg_call + st.nbytes
     peak, peak_kind = hbm_peak()
-    line = {
-        "metric": "decode block_step latency (p50) and tokens*heads/s", "value": job_throughput(units, world, p50 * 1e-3),
-        "unit": "tokens*heads/s", "n_gpus": world, "steps": reps * nb, "warmup": max(1, args.warmup // 5) * nb,
-        "ms_per_step": p50 * 1e-3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": f"{w.name}: {nb} block_step calls of {F}x{w.Hg}x{w.Wg} tokens, B={w.B} H={w.H} d={w.d} "
-                               f"{w.dtype}, commit=1, per-block latency from CUDA events around each call; "
-                               f"{len(distinct)} distinct seeded blocks cycled",
-                   "l2": "per-block inputs (63 MB) live in HBM; no flush", "parallelism": f"independent replica per GPU x{world}"},
-        "latency_us": {"p50": p50, "p99": p99, "min": float(lat.min()), "max": float(lat.max()),
-                       "host_enqueue_per_block": host_us, "graph_replay_per_block": graph_us,
-                       "graph_error": graph_err},
-        "roofline": {"bound": "hbm", "kernel": "block_step (3 launches)", "achieved": alg / (p50 * 1e-6) / 1e9,
-                     "peak": peak, "unit": "GB/s", "frac": alg / (p50 * 1e-6) / 1e9 / peak,
-                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": None, "algorithmic_bytes_per_launch": alg},
+    per_block_us = graph_us if graph_us is not None else p50
+    rec = {
+        "workload": f"{w.name}: {nb} blocks of {F}x{w.Hg}x{w.Wg} tokens, B={w.B} H={w.H} d={w.d} {w.dtype}, "
+                    + (f"each block {denoise_steps} read-only block steps (commit=0, fresh Q/K/V) then one commit"
+                       if denoise_steps else "one block_step (commit=1) per block")
+                    + f"; {ndist} distinct seeded inputs cycled",
+        "calls_per_block": calls_per_block,
+        "latency_us_per_block": {"p50": p50, "p99": p99, "min": float(lat.min()), "max": float(lat.max()),
+                                 "graph_replay": graph_us, "graph_error": graph_err,
+                                 "host_enqueue": host_us},
+        "latency_us_per_call_graph": None if graph_us is None else graph_us / calls_per_block,
+        "value": job_throughput(units * calls_per_block, world, per_block_us * 1e-3), "unit": UNIT,
+        "roofline": {"bound": "hbm", "kernel": "block step (all launches)", "achieved": alg_block / (per_block_us * 1e-6) / 1e9,
+                     "peak": peak, "unit": "GB/s", "frac": alg_block / (per_block_us * 1e-6) / 1e9 / peak,
+                     "peak_source": f"{peak_kind} hbm_gbs", "timing": "graph replay" if graph_us is not None else "p50",
+                     "algorithmic_bytes_per_block": alg_block},
         "state_bytes": st.nbytes, "device_memory_flat": bool(mem_flat),
-        "clocks": clk.summary(),
     }
+    st.free()
+    return rec
+
+
+def run_blin(args):
+    torch, blin, world, rank, local = _load_blin(args)
+    main_name = "720p" if args.config == "all" else args.config
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)  # let the sampler start
+        if main_name in ("decode", "denoise"):
+            w = workloads.CONFIGS["decode"]
+            rec = measure_decode(args, w, torch, blin, world, rank, clk, 4 if main_name == "denoise" else 0)
+            main = {"metric": "decode block_step tokens*heads/s (graph-replayed blocks)", "value": rec["value"],
+                    "ms_per_step": rec["latency_us_per_block"]["p50"] * 1e-3, "roofline": rec["roofline"],
+                    "config": {"workload": rec["workload"], "parallelism": f"independent replica per GPU x{world}",
+                               "l2": "per-block inputs live in HBM; no flush"}, "decode": rec}
+        else:
+            w = workloads.CONFIGS[main_name]
+            rec = measure_prefill(args, w, torch, blin, world, rank, clk, full=True)
+            main = {"metric": METRIC, "value": rec["value"], "ms_per_step": rec["ms_per_step"],
+                    "config": config_dict(w, world)}
+            for key in ("path", "hbm_gbs_whole_step", "hbm_frac_whole_step", "kernel_ms", "roofline", "e2e",
+                        "gpu_launches", "cpu_baseline"):
+                if key in rec:
+                    main[key] = rec[key]
+        subs = {}
+        if args.config == "all" and not args.no_sub_records:
+            for name in ("480p", "wide"):
+                subs[name] = measure_prefill(args, workloads.CONFIGS[name], torch, blin, world, rank, clk, full=False)
+            subs["decode"] = measure_decode(args, workloads.CONFIGS["decode"], torch, blin, world, rank, clk, 0)
+            subs["denoise"] = measure_decode(args, workloads.CONFIGS["decode"].with_(steps=16), torch, blin, world,
+                                             rank, clk, 4)
+        time.sleep(0.25)
+    line = {"metric": main.pop("metric"), "value": main.pop("value"), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": main.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": workloads.CONFIGS[
+                "decode" if main_name in ("decode", "denoise") else main_name].dtype, "data": "synthetic"}
+    line.update(main)
+    line["clocks"] = clk.summary()
+    if subs:
+        line["sub_records"] = subs
     if rank == 0:
         print(json.dumps(line), flush=True)
-    st.free()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -608,23 +643,24 @@ def run_decode(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)  # ~0.5 s timed: the 200 ms clock sampler sees load
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="blin", choices=["blin", "reference"])
-    ap.add_argument("--config", default="480p", choices=["480p", "720p", "wide", "decode"])
-    ap.add_argument("--cpu-rows", type=int, default=2000, help="oracle rows for the CPU baseline (about 10 s)")
+    ap.add_argument("--config", default="all", choices=["all", "480p", "720p", "wide", "decode", "denoise"],
+                    help="all: the 720p headline plus 480p, wide, decode and denoise sub-records")
+    ap.add_argument("--cpu-rows", type=int, default=None,
+                    help="oracle rows for the CPU baseline (default: scaled to about 10-20 s)")
     ap.add_argument("--ref-rows", type=int, default=None,
                     help="oracle rows per reference-arm step (default: sized so the whole run stays near a minute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-records", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=7, help="head chunks pipelined through the e2e step")
     args = ap.parse_args()
-    w = workloads.CONFIGS[args.config]
     if args.impl == "reference":
-        run_reference(args, w)
-    elif args.config == "decode":
-        run_decode(args, w)
+        name = "720p" if args.config == "all" else args.config
+        run_reference(args, workloads.CONFIGS["decode" if name == "denoise" else name])
     else:
-        run_blin(args, w)
+        run_blin(args)
 
 
 if __name__ == "__main__":

@@ -22,7 +22,7 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 __all__ = ["BlinError", "BlockState", "prefill", "block_step", "workspace_size", "device_status",
-           "LaunchTimer", "KERNELS", "lib", "LIB_PATH", "F32", "BF16"]
+           "last_path", "LaunchTimer", "KERNELS", "lib", "LIB_PATH", "F32", "BF16"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libblin.so")
@@ -63,7 +63,9 @@ def _load() -> ctypes.CDLL:
     L.blin_prefill_workspace_size.argtypes = [I, I, I, ctypes.POINTER(Geom)]
     L.blin_prefill_workspace_size.restype = S
     L.blin_prefill.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), P, P, S, P]
-    L.blin_block_step.argtypes = [P, P, P, P, I, I, I, I, I, I, I, ctypes.POINTER(I * 3), F, F, P, I, P]
+    L.blin_block_step.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), P, I, P]
+    L.blin_last_path.argtypes = []
+    L.blin_last_path.restype = I
     L.blin_last_error.restype = ctypes.c_char_p
     L.blin_device_status.argtypes = [ctypes.POINTER(I)]
     L.blin_version.restype = ctypes.c_char_p
@@ -220,25 +222,38 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Sequence[in
 
 def block_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Hg: int, Wg: int, frames: int,
                rope_split: Sequence[int], state: BlockState, theta: float = 1e4, eps: float = 1e-6,
-               commit: bool = True, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+               commit: bool = True, out: Optional[torch.Tensor] = None, stream=None,
+               block_frames: Optional[int] = None) -> torch.Tensor:
     """One autoregressive block of `frames` latent frames read against (and, if
-    commit, added to) the cached state."""
+    commit, added to) the cached state.  `block_frames` is the causal block
+    length F (default: `frames`); the call's frames must lie in one block."""
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
     if N != frames * Hg * Wg:
         raise ValueError(f"N={N} but frames*Hg*Wg={frames * Hg * Wg}")
     if out is None:
         out = torch.empty_like(q)
-    split = (ctypes.c_int * 3)(*[int(x) for x in rope_split])
+    g = _geom(frames, Hg, Wg, frames if block_frames is None else block_frames, rope_split, theta, eps)
     _check(lib.blin_block_step(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
                                ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-                               _dtype_code(q), B, H, d, int(Hg), int(Wg), int(frames),
-                               ctypes.byref(split), float(theta), float(eps), state.handle,
+                               _dtype_code(q), B, H, d, ctypes.byref(g), state.handle,
                                1 if commit else 0, _stream(stream)))
     return out
 
 
+PATHS = {0: "none", 1: "tensor_core", 2: "cuda_core"}
+
+
+def last_path() -> str:
+    """Which kernels this thread's last prefill / block_step ran: "tensor_core" or "cuda_core"."""
+    return PATHS[int(lib.blin_last_path())]
+
+
 KERNELS = ("rope_table", "partial_states", "block_scan", "output")
+# Algorithmic HBM bytes of each launch per token*head, in units of d * element size:
+# pass 1 reads K and V, pass 2 reads Q and writes O; the scan and the table move no
+# per-token bytes (None: not a roofline candidate).
+KERNEL_BYTES_PER_UNIT = {"rope_table": None, "partial_states": 2, "block_scan": None, "output": 2}
 
 
 class LaunchTimer:

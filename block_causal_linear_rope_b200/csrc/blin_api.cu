@@ -27,9 +27,11 @@ struct blin_state {
     int t_next;
     void *scratch;  // block-step workspace (tables, partials, prefix)
     size_t scratch_bytes;
+    cudaEvent_t last_use;  // recorded after every call that reads or writes S, z or the scratch
 };
 
 static thread_local char g_err[512] = "";
+static thread_local int g_last_path = 0;  // blin_path of this thread's last call that launched kernels
 
 static blin_status fail(blin_status st, const char *fmt, ...) {
     va_list ap;
@@ -167,6 +169,35 @@ static void plan_bind(Plan &p, void *ws) {
     p.g.prefix = reinterpret_cast<float *>(base + p.tab_bytes + p.part_bytes);
 }
 
+// ---------------------------------------------------------------- contexts
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+unsigned long long blin::current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS) return 0;
+    if (ctx == nullptr) {  // no context yet: let the runtime bind the device's primary one
+        cudaFree(nullptr);
+        if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    }
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
 // ---------------------------------------------------------------- TMA descriptors
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -223,6 +254,7 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
     const KGeom &g = p.g;
     const int d = p.d;
     const bool tc = dt == BLIN_BF16 && tc_supported(d, split) && g.tab_smem;
+    g_last_path = tc ? BLIN_PATH_TENSOR_CORE : BLIN_PATH_CUDA_CORE;
     CUtensorMap mq, mk, mv, mo;
     if (tc) {
         const long long rows = (long long)g.BH * g.N;
@@ -257,6 +289,18 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
     g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(3, true, s);
     return BLIN_OK;
+}
+
+// Records the state's last-use event on `s` (blin_state_free waits for it).
+// Work captured into a CUDA graph is not marked: it runs when the graph is
+// launched, which the library does not see.
+static blin_status mark_state_use(blin_state *st, cudaStream_t s) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "stream capture query");
+    if (cap != cudaStreamCaptureStatusNone) return BLIN_OK;
+    e = cudaEventRecord(st->last_use, s);
+    return e == cudaSuccess ? BLIN_OK : cuda_fail(e, "state event record");
 }
 
 static blin_status check_state(const blin_state *st) {
@@ -300,9 +344,12 @@ blin_status blin_state_init(int B, int H, int d, blin_stream stream, blin_state 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(st->S, 0, sb, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(st->z, 0, zb, s);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st->last_use, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(st->last_use, s);
     if (e != cudaSuccess) {
         if (st->S) cudaFree(st->S);
         if (st->z) cudaFree(st->z);
+        if (st->last_use) cudaEventDestroy(st->last_use);
         delete st;
         return cuda_fail(e, "state allocation");
     }
@@ -316,14 +363,16 @@ blin_status blin_state_free(blin_state *st) {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(st->device);
-    cudaError_t e = cudaDeviceSynchronize();
+    // wait only for the work that used this state (its last call's stream position)
+    cudaError_t e = cudaEventSynchronize(st->last_use);
+    cudaEventDestroy(st->last_use);
     cudaFree(st->S);
     cudaFree(st->z);
     if (st->scratch) cudaFree(st->scratch);
     cudaSetDevice(prev);
     st->magic = kFreedMagic;
     delete st;
-    if (e != cudaSuccess) return cuda_fail(e, "synchronise before state free");
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the state's last use before freeing it");
     return BLIN_OK;
 }
 
@@ -336,6 +385,7 @@ blin_status blin_state_reset(blin_state *st, blin_stream stream) {
     cudaError_t e = cudaMemsetAsync(st->S, 0, sb, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(st->z, 0, zb, s);
     if (e != cudaSuccess) return cuda_fail(e, "state reset");
+    if ((rc = mark_state_use(st, s)) != BLIN_OK) return rc;
     st->t_next = 0;
     return BLIN_OK;
 }
@@ -366,7 +416,7 @@ blin_status blin_state_copy_to_host(const blin_state *st, void *host, size_t byt
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(static_cast<char *>(host) + sb, st->z, bytes - sb, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return cuda_fail(e, "state copy to host");
-    return BLIN_OK;
+    return mark_state_use(const_cast<blin_state *>(st), s);
 }
 
 blin_status blin_state_copy_from_host(blin_state *st, const void *host, size_t bytes, int t_next,
@@ -383,6 +433,7 @@ blin_status blin_state_copy_from_host(blin_state *st, const void *host, size_t b
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(st->z, static_cast<const char *>(host) + sb, bytes - sb, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "state copy from host");
+    if ((rc = mark_state_use(st, s)) != BLIN_OK) return rc;
     st->t_next = t_next;
     return BLIN_OK;
 }
@@ -443,16 +494,21 @@ blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, b
     rc = run(p, q, k, v, o, dt, st ? st->S : nullptr, st ? st->z : nullptr, st ? st->S : nullptr,
              st ? st->z : nullptr, (double)g->theta, g->rope_split, static_cast<cudaStream_t>(stream));
     if (rc != BLIN_OK) return rc;
-    if (st) st->t_next += g->T;
+    if (st) {
+        if ((rc = mark_state_use(st, static_cast<cudaStream_t>(stream))) != BLIN_OK) return rc;
+        st->t_next += g->T;
+    }
     return BLIN_OK;
 }
 
 blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
-                            int H, int d, int Hgt, int Wid, int frames, const int rope_split[3],
-                            float theta, float eps, blin_state *st, int commit, blin_stream stream) {
-    blin_status rc = check_common(B, H, d, frames, Hgt, Wid, rope_split, theta, eps);
+                            int H, int d, const blin_geom *g, blin_state *st, int commit, blin_stream stream) {
+    if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
+    blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;
-    if (frames < 1) return fail(BLIN_ERR_INVALID_ARG, "frames must be >= 1");
+    const int frames = g->T, F = g->block_frames;
+    if (frames < 1) return fail(BLIN_ERR_INVALID_ARG, "frames (geom T) must be >= 1");
+    if (F < 1) return fail(BLIN_ERR_INVALID_ARG, "block_frames must be >= 1");
     if (commit != 0 && commit != 1) return fail(BLIN_ERR_INVALID_ARG, "commit must be 0 or 1");
     if ((rc = check_io(q, k, v, o, dt)) != BLIN_OK) return rc;
     if ((rc = check_state(st)) != BLIN_OK) return rc;
@@ -460,16 +516,24 @@ blin_status blin_block_step(const void *q, const void *k, const void *v, void *o
         return fail(BLIN_ERR_STATE, "state is B=%d H=%d d=%d, call is B=%d H=%d d=%d", st->B, st->H, st->d,
                     B, H, d);
     if ((long long)st->t_next + frames >= (1LL << 30)) return fail(BLIN_ERR_SHAPE, "frame index overflow");
+    // one causal block per call: the frames [t_next, t_next + frames) share block t_next / F
+    if (st->t_next % F + frames > F)
+        return fail(BLIN_ERR_SHAPE,
+                    "frames [%d, %d) cross a block boundary (block_frames %d): a block step covers one block",
+                    st->t_next, st->t_next + frames, F);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    Plan p = make_plan(B, H, d, frames, Hgt, Wid, frames, st->t_next, true, rope_split, eps);
+    Plan p = make_plan(B, H, d, frames, g->Hgt, g->Wid, frames, st->t_next, true, g->rope_split, g->eps);
     if ((rc = ensure_scratch(st, plan_bytes(p), s)) != BLIN_OK) return rc;
     plan_bind(p, st->scratch);
     rc = run(p, q, k, v, o, dt, st->S, st->z, commit ? st->S : nullptr, commit ? st->z : nullptr,
-             (double)theta, rope_split, s);
+             (double)g->theta, g->rope_split, s);
     if (rc != BLIN_OK) return rc;
+    if ((rc = mark_state_use(st, s)) != BLIN_OK) return rc;
     if (commit) st->t_next += frames;
     return BLIN_OK;
 }
+
+int blin_last_path(void) { return g_last_path; }
 
 blin_status blin_set_timing_events(void *const *events, int n) {
     if (events != nullptr && n < 8) return fail(BLIN_ERR_INVALID_ARG, "need 8 events (got %d)", n);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/blin.h"
 
 namespace blin {
@@ -76,7 +78,7 @@ cudaError_t launch_output_simt(const KGeom &g, int d, bool bf16, const void *q, 
                                cudaStream_t s);
 // Tensor-core path (bf16, d in {32, 64}, splits with a compiled variant).
 bool tc_supported(int d, const int split[3]);
-// Partial states plus the fused per-head scan (writes prefix and S_out/z_out).
+// Chunk partial states (the block scan follows as its own launch).
 cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv,
                               cudaStream_t s);
 // Shared-memory bytes the tensor-core kernels need for a RoPE table copy of
@@ -87,6 +89,45 @@ cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const
 
 // Device watchdog access.
 cudaError_t read_and_clear_watchdog(int *code);
+
+// Unique id of the calling thread's current CUDA context (0 if none or the
+// driver cannot tell).  Device addresses and function attributes belong to a
+// context, so per-context caches key on this, not on the device ordinal: a
+// host framework may make another context current, and cudaDeviceReset
+// replaces the primary one.
+unsigned long long current_context_id();
+
+// A small cache of per-context values (device addresses, flags), keyed by
+// current_context_id(); thread safe.
+template <typename V>
+struct ContextCache {
+    static constexpr int kSlots = 32;
+    std::mutex mu;
+    unsigned long long key[kSlots] = {};
+    V val[kSlots] = {};
+    int next = 0;
+    bool get(unsigned long long k, V *out) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < kSlots; ++i)
+            if (key[i] == k && k != 0) {
+                *out = val[i];
+                return true;
+            }
+        return false;
+    }
+    void put(unsigned long long k, V v) {
+        if (k == 0) return;
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < kSlots; ++i)
+            if (key[i] == k) {
+                val[i] = v;
+                return;
+            }
+        key[next] = k;
+        val[next] = v;
+        next = (next + 1) % kSlots;
+    }
+};
 
 // Records `msg` as this thread's blin_last_error() text and returns `st`.
 blin_status set_last_error(blin_status st, const char *msg);

@@ -1,5 +1,8 @@
-// All device code of libblin lives in this translation unit (one watchdog word
-// per device, no relocatable device code needed) together with its launchers.
+// Device code of libblin's attention path and its launchers.  Besides the
+// kernels, this translation unit holds the one device-resident watchdog word
+// (g_watchdog); the only other device-resident object of the library is
+// blin_prefill_static's scratch array in blin_noalloc.cu.  Host code reaches
+// both through cudaGetSymbolAddress, so no relocatable device code is needed.
 #include <cuda_bf16.h>
 
 #include <utility>
@@ -23,16 +26,16 @@ cudaError_t read_and_clear_watchdog(int *code) {
 }
 
 static int *watchdog_ptr() {
-    // Address of this device's watchdog word (cached per device).
-    static int *ptrs[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (ptrs[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_watchdog) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<int *>(p);
-    }
-    return ptrs[dev];
+    // Address of the current context's watchdog word (a module's device
+    // variables exist once per context).
+    static ContextCache<int *> cache;
+    const unsigned long long ctx = current_context_id();
+    int *p = nullptr;
+    if (cache.get(ctx, &p)) return p;
+    void *a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_watchdog) != cudaSuccess) return nullptr;
+    cache.put(ctx, static_cast<int *>(a));
+    return static_cast<int *>(a);
 }
 
 cudaError_t launch_rope_table(const KGeom &g, cudaStream_t s) {
@@ -96,20 +99,19 @@ bool tc_supported(int d, const int split[3]) {
     return false;
 }
 
-// Raise the dynamic shared-memory limit of a kernel (cached per device and
-// kernel: the template parameter is the kernel itself, not its type).
+// Raise the dynamic shared-memory limit of a kernel (once per context and
+// kernel: function attributes belong to a context; the template parameter is
+// the kernel itself, not its type).
 template <auto Kernel>
 static cudaError_t set_smem(int bytes) {
-    static int done[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
-    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    // the largest shared-memory carveout, so that two CTAs of ~113 KB fit on an SM
+    static ContextCache<int> done;
+    const unsigned long long ctx = current_context_id();
+    int have = 0;
+    if (done.get(ctx, &have) && have >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 227 * 1024;
+    if (e == cudaSuccess) done.put(ctx, 227 * 1024);
     return e;
 }
 

@@ -7,7 +7,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/blin.h"
 #include "blin_internal.cuh"
@@ -21,36 +20,32 @@ constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
 // process exits, and every call on that GPU shares it.
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-// Device address of g_static_scratch, looked up once per device.  In host
-// code the array's name is only a host-side stand-in, so the address must come
-// from cudaGetSymbolAddress with that device current.
-constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
-std::mutex g_scratch_mu;
+// Device address of g_static_scratch in each CUDA context.  In host code the
+// array's name is only a host-side stand-in, so the address must come from
+// cudaGetSymbolAddress with that context current.  A module's device variables
+// exist once per context (not once per device ordinal): a host framework may
+// make a context of its own current, and cudaDeviceReset replaces the primary
+// context, so the cache is keyed by the context's unique id.
+blin::ContextCache<void *> g_scratch_addr;
 
-blin_status scratch_for_current_device(void **out, char *msg, size_t msg_len) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        snprintf(msg, msg_len, "cudaGetDevice: %s", cudaGetErrorString(e));
+blin_status scratch_for_current_context(void **out, char *msg, size_t msg_len) {
+    const unsigned long long ctx = blin::current_context_id();
+    if (ctx == 0) {
+        snprintf(msg, msg_len, "no CUDA context is current (or the driver cannot name it)");
         return BLIN_ERR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) {
-        snprintf(msg, msg_len, "device %d is beyond the %d devices this entry point supports", dev, kMaxDevices);
-        return BLIN_ERR_INVALID_ARG;
+    void *p = nullptr;
+    if (g_scratch_addr.get(ctx, &p)) {
+        *out = p;
+        return BLIN_OK;
     }
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess || p == nullptr) {
-            snprintf(msg, msg_len, "cudaGetSymbolAddress(static scratch) on device %d: %s", dev,
-                     cudaGetErrorString(e));
-            return BLIN_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = p;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+        snprintf(msg, msg_len, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+        return BLIN_ERR_CUDA;
     }
-    *out = g_scratch_addr[dev];
+    g_scratch_addr.put(ctx, p);
+    *out = p;
     return BLIN_OK;
 }
 
@@ -77,7 +72,7 @@ blin_status blin_prefill_static(const void *q, const void *k, const void *v, voi
         return blin::set_last_error(BLIN_ERR_WORKSPACE, msg);
     }
     void *scratch = nullptr;
-    const blin_status rc = scratch_for_current_device(&scratch, msg, sizeof msg);
+    const blin_status rc = scratch_for_current_context(&scratch, msg, sizeof msg);
     if (rc != BLIN_OK) return blin::set_last_error(rc, msg);
     return blin_prefill(q, k, v, o, dt, B, H, d, g, st, scratch, kStaticScratchBytes, stream);
 }

@@ -96,7 +96,11 @@ typedef struct blin_state blin_state; /* opaque (S, z) cache on one device */
  * it (talk transcript: constant KV-cache memory for any video length). */
 BLIN_API blin_status blin_state_init(int B, int H, int d, blin_stream stream, blin_state **out);
 
-/* Free the cache and its scratch (synchronises the device).  NULL is a no-op. */
+/* Free the cache and its scratch.  Waits for the last call that used the state
+ * (on whatever stream it ran) to finish first; other work on the device is not
+ * waited for.  Calls captured into a CUDA graph are not tracked: the caller
+ * must let every launch of such a graph finish before freeing the state.
+ * NULL is a no-op. */
 BLIN_API blin_status blin_state_free(blin_state *st);
 
 /* Zero S and z (on stream) and set t_next = 0. */
@@ -150,22 +154,26 @@ BLIN_API blin_status blin_prefill(const void *q, const void *k, const void *v, v
 
 /* ---------------------------------------------------------------- decode */
 
-/* One autoregressive block (talk transcript, block-causal walk-through: the
- * new block reads the cached state plus its own contribution; the sum is
- * cached for the next block).
- *   q, k, v, o  device [B][H][frames*Hgt*Wid][d] of dtype dt
- *   frames      latent frames in this block, 1..block_frames of the caller's
- *               schedule (the library treats the whole call as one block)
- *   commit      1: S += block K~^T V, z += sum phi(k), t_next += frames.
+/* One autoregressive block, or the part of one that is ready (talk
+ * transcript, block-causal walk-through: the new block reads the cached state
+ * plus its own contribution; the sum is cached for the next block).
+ *   q, k, v, o  device [B][H][g->T * g->Hgt * g->Wid][d] of dtype dt
+ *   g           g->T = latent frames of this call (>= 1), g->block_frames = F,
+ *               the causal block length; rope_split, theta, eps as for prefill
+ *   commit      1: S += the call's K~^T V, z += sum phi(k), t_next += T.
  *               0: read-only pass (a denoising step of the same block);
  *                  the cache is left unchanged.
- * Positions continue from the cache: t_abs = t_next + t.  Needs scratch owned
+ * Positions continue from the cache: t_abs = t_next + t.  The call's frames
+ * must lie in one causal block: (t_next % F) + T <= F, else BLIN_ERR_SHAPE
+ * (a call that would cross a block boundary is rejected, never regrouped).
+ * A call that starts a block and covers it whole reduces its keys exactly as
+ * blin_prefill does, so a block-by-block stream gives bitwise the outputs and
+ * the final (S, z) of one prefill over the same frames.  Needs scratch owned
  * by the state; the first call with a larger block grows it (allocation on
  * stream), blin_state_reserve avoids that. */
 BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
-                            int B, int H, int d, int Hgt, int Wid, int frames,
-                            const int rope_split[3], float theta, float eps,
-                            blin_state *st, int commit, blin_stream stream);
+                            int B, int H, int d, const blin_geom *g, blin_state *st, int commit,
+                            blin_stream stream);
 
 /* ---------------------------------------------------------------- no allocation */
 
@@ -180,14 +188,17 @@ BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v
  * holds it until the process exits, and nothing is allocated per call.
  *   - Shapes whose blin_prefill_workspace_size exceeds the capacity are
  *     rejected with BLIN_ERR_WORKSPACE and a message naming both sizes.
- *   - The first call on each device looks up the scratch area's device
- *     address (cudaGetSymbolAddress with that device current); make that
- *     first call before any stream capture.
+ *   - The first call in each CUDA context (normally one per device: the
+ *     primary context) looks up the scratch area's device address
+ *     (cudaGetSymbolAddress with that context current) and caches it under
+ *     the context's unique id; make that first call before any stream capture.
+ *     Another context made current later, or a new primary context after
+ *     cudaDeviceReset, gets its own lookup.
  *   - All calls on a device share the one scratch area and it keeps the last
  *     call's contents.  Nothing in it needs to start at zero (each call writes
  *     everything it reads), but calls that overlap on the GPU, e.g. on two
  *     streams at once, race on it: serialise them.
- *   - Results are those of blin_prefill on the same arguments. */
+ *   - Results are those of blin_prefill on the same arguments, bit for bit. */
 BLIN_API blin_status blin_prefill_static(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                                          int B, int H, int d, const blin_geom *g, blin_state *st,
                                          blin_stream stream);
@@ -199,6 +210,15 @@ BLIN_API size_t blin_prefill_static_capacity(void);
 
 /* Thread-local message for the last non-OK status of this thread ("" if none). */
 BLIN_API const char *blin_last_error(void);
+
+/* Which kernels this thread's last blin_prefill / blin_block_step that
+ * launched any ran (a call rejected before launch leaves it unchanged):
+ *   BLIN_PATH_TENSOR_CORE  bf16 storage with a compiled RoPE split whose
+ *                          RoPE table fits shared memory: tcgen05/TMA kernels
+ *   BLIN_PATH_CUDA_CORE    otherwise (fp32 storage, other splits): fp32 FMA
+ *                          kernels.  Both compute the same function. */
+typedef enum { BLIN_PATH_NONE = 0, BLIN_PATH_TENSOR_CORE = 1, BLIN_PATH_CUDA_CORE = 2 } blin_path;
+BLIN_API int blin_last_path(void);
 
 /* Read (synchronously) and clear the current device's kernel watchdog word:
  * 0 = no bounded wait ran out since the last call; otherwise a code naming the

@@ -100,23 +100,31 @@ def test_prefill_with_no_frames_is_a_no_op():
 
 def test_geom_null_and_state_null():
     assert blin.lib.blin_prefill(FAKE, FAKE, FAKE, FAKE, 1, 1, 2, 32, None, None, FAKE, 1 << 20, None) == INVALID
-    split = (ctypes.c_int * 3)(8, 12, 12)
-    rc = blin.lib.blin_block_step(FAKE, FAKE, FAKE, FAKE, 1, 1, 2, 32, 4, 4, 3, ctypes.byref(split), 1e4, 1e-6,
-                                  None, 1, None)
-    assert rc == INVALID
+    assert blin.lib.blin_block_step(FAKE, FAKE, FAKE, FAKE, 1, 1, 2, 32, None, None, 1, None) == INVALID
+    g = geom(T=3, Hg=4, Wg=4)
+    assert blin.lib.blin_block_step(FAKE, FAKE, FAKE, FAKE, 1, 1, 2, 32, ctypes.byref(g), None, 1, None) == INVALID
 
 
 def test_block_step_argument_checks():
-    split = (ctypes.c_int * 3)(8, 12, 12)
-    bad = (ctypes.c_int * 3)(8, 12, 14)
-    call = lambda **kw: blin.lib.blin_block_step(
-        kw.get("q", FAKE), FAKE, FAKE, FAKE, kw.get("dt", 1), 1, 2, kw.get("d", 32), 4, 4, kw.get("frames", 3),
-        ctypes.byref(kw.get("split", split)), 1e4, 1e-6, FAKE, kw.get("commit", 1), None)
+    def call(**kw):
+        g = geom(T=kw.get("frames", 3), Hg=4, Wg=4, F=kw.get("F", 3), split=kw.get("split", (8, 12, 12)))
+        return blin.lib.blin_block_step(kw.get("q", FAKE), FAKE, FAKE, FAKE, kw.get("dt", 1), 1, 2, kw.get("d", 32),
+                                        ctypes.byref(g), FAKE, kw.get("commit", 1), None)
     assert call(frames=0) == INVALID
-    assert call(split=bad) == SHAPE
+    assert call(F=0) == INVALID
+    assert call(split=(8, 12, 14)) == SHAPE
     assert call(commit=2) == INVALID
     assert call(dt=5) == DTYPE
     assert call(q=FAKE + 2) == ALIGN
+
+
+def test_last_path_starts_empty():
+    import threading
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(blin.lib.blin_last_path()))
+    t.start()
+    t.join()
+    assert seen == [0]  # thread-local: a fresh thread has run nothing
 
 
 def test_state_accessors_reject_null():

@@ -49,7 +49,7 @@ def test_tiny_streamed_equals_prefill_bitwise(blin, dtype):
     for (f0, f1) in w.block_frame_ranges():
         qb, kb, vb = workloads.call_tensors(w.with_(t0=f0, T=f1 - f0))
         ob = blin.block_step(dev(qb, dtype), dev(kb, dtype), dev(vb, dtype), w.Hg, w.Wg, f1 - f0, w.split,
-                             st_b, theta=w.theta, eps=w.eps)
+                             st_b, theta=w.theta, eps=w.eps, block_frames=w.F)
         outs.append(host(ob))
     streamed = np.concatenate(outs, axis=2)
     np.testing.assert_array_equal(streamed, full)
@@ -96,6 +96,7 @@ def test_unsupported_split_runs_on_cuda_cores(blin):
     w = workloads.Workload("split", B=1, H=2, d=32, dtype="bf16", T=6, Hg=4, Wg=9, F=2, split=(16, 8, 8), seed=3)
     q, k, v = workloads.call_tensors(w)
     got = run_prefill(blin, w, q, k, v).reshape(-1, w.N, w.d)
+    assert blin.last_path() == "cuda_core"
     ref, _, _ = oracle_all_rows(w, q, k, v)
     assert rel_err(got, ref) <= TOL["bf16"]
 
@@ -249,13 +250,15 @@ def test_minute_long_decode(blin):
         wb = w.with_(T=3, t0=3 * blk_i)
         q, k, v = workloads.call_tensors(wb)
         o = blin.block_step(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), w.Hg, w.Wg, 3, w.split, st,
-                            theta=w.theta, eps=w.eps)
+                            theta=w.theta, eps=w.eps, block_frames=w.F)
         got = host(o)[0, heads]
         del o
         torch.cuda.synchronize()
-        mem = torch.cuda.memory_allocated()
+        # free device memory as the driver sees it: counts the library's own
+        # allocations (state, scratch), which PyTorch's allocator statistics do not
+        mem = torch.cuda.mem_get_info()[0]
         mem0 = mem if mem0 is None else mem0
-        assert mem == mem0, "device memory grew during decode"
+        assert mem == mem0, "device memory changed during decode"
         sub = lambda x: np.ascontiguousarray(x[0, heads])
         ref, S_o, z_o = oracle.recurrence(sub(q), sub(k), sub(v), *oracle.grid(3, w.Hg, w.Wg, w.F, 3 * blk_i),
                                           w.split, w.theta, w.eps, S_o, z_o)
@@ -268,3 +271,102 @@ def test_minute_long_decode(blin):
     S, z = st.to_host()
     assert rel_err(S.numpy()[0, heads], S_o) <= 5e-3
     assert rel_err(z.numpy()[0, heads], z_o) <= 1e-5
+
+
+# --------------------------------------------------------------------------- bitwise streaming, multi-chunk blocks
+def _stream_blocks(blin, w, qd, kd, vd, st):
+    """Feed a prefill-shaped call block by block through block_step; returns the concatenated output."""
+    outs = []
+    for (f0, f1) in w.block_frame_ranges():
+        n0, n1 = (f0 - w.t0) * w.HW, (f1 - w.t0) * w.HW
+        outs.append(blin.block_step(qd[:, :, n0:n1].contiguous(), kd[:, :, n0:n1].contiguous(),
+                                    vd[:, :, n0:n1].contiguous(), w.Hg, w.Wg, f1 - f0, w.split, st,
+                                    theta=w.theta, eps=w.eps, block_frames=w.F))
+    return torch.cat(outs, dim=2)
+
+
+@pytest.mark.parametrize("name", ["480p", "wide"])
+def test_full_size_streamed_equals_prefill_bitwise(blin, name):
+    """Every block of the workload through block_step == one prefill, bit for bit (O, S, z).
+
+    480p blocks are 4,680 tokens (several state chunks per block, reduced in a
+    fixed order); the block steps also use smaller output groups than the
+    prefill, which must not change any output bit.
+    """
+    w = workloads.CONFIGS[name]
+    q, k, v = workloads.call_tensors(w)
+    qd, kd, vd = dev(q, w.dtype), dev(k, w.dtype), dev(v, w.dtype)
+    st_a = blin.BlockState(w.B, w.H, w.d)
+    full = blin.prefill(qd, kd, vd, (w.T, w.Hg, w.Wg), w.F, w.split, w.theta, w.eps, state=st_a)
+    assert blin.last_path() == "tensor_core"
+    st_b = blin.BlockState(w.B, w.H, w.d)
+    streamed = _stream_blocks(blin, w, qd, kd, vd, st_b)
+    assert blin.last_path() == "tensor_core"
+    torch.cuda.synchronize()
+    assert torch.equal(streamed, full), "streamed block outputs differ from the prefill"
+    Sa, za = st_a.to_host()
+    Sb, zb = st_b.to_host()
+    assert torch.equal(Sa, Sb) and torch.equal(za, zb), "streamed cache differs from the prefill's"
+    assert st_a.t_next == st_b.t_next == w.T
+
+
+def test_decode_block_through_prefill_state_bitwise(blin):
+    """Prefill 3 decode-sized blocks into a cache, then block_step the 4th: the 4th block's rows
+    and the final cache equal a one-shot prefill of all 4 blocks, bit for bit."""
+    w = workloads.CONFIGS["decode"].with_(T=12, steps=1)
+    q, k, v = workloads.call_tensors(w)
+    qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+    st_full = blin.BlockState(w.B, w.H, w.d)
+    full = blin.prefill(qd, kd, vd, (w.T, w.Hg, w.Wg), w.F, w.split, w.theta, w.eps, state=st_full)
+    n3 = 9 * w.HW
+    st = blin.BlockState(w.B, w.H, w.d)
+    head = blin.prefill(qd[:, :, :n3].contiguous(), kd[:, :, :n3].contiguous(), vd[:, :, :n3].contiguous(),
+                        (9, w.Hg, w.Wg), w.F, w.split, w.theta, w.eps, state=st)
+    last = blin.block_step(qd[:, :, n3:].contiguous(), kd[:, :, n3:].contiguous(), vd[:, :, n3:].contiguous(),
+                           w.Hg, w.Wg, 3, w.split, st, theta=w.theta, eps=w.eps, block_frames=w.F)
+    torch.cuda.synchronize()
+    assert torch.equal(head, full[:, :, :n3])
+    assert torch.equal(last, full[:, :, n3:])
+    S1, z1 = st.to_host()
+    S2, z2 = st_full.to_host()
+    assert torch.equal(S1, S2) and torch.equal(z1, z2)
+    # and the rows agree with the oracle
+    ref, _, _ = oracle_all_rows(w, q, k, v)
+    assert rel_err(host(full).reshape(-1, w.N, w.d), ref) <= TOL["bf16"]
+
+
+def test_block_step_after_prefill_ending_mid_block(blin):
+    """A prefill that stops inside a block, then block steps that finish it and go on.
+
+    The block length is part of the call: a step whose frames would cross a
+    block boundary is rejected (BLIN_ERR_SHAPE), the state untouched.  Steps
+    that finish the open block see the whole block (cache + own frames), so
+    their rows equal the one-shot rows; the final cache equals the one-shot one.
+    """
+    w = workloads.Workload("mid", B=1, H=4, d=32, dtype="bf16", T=9, Hg=12, Wg=20, F=3, split=(8, 12, 12), seed=13)
+    q, k, v = workloads.call_tensors(w)
+    ref, S_ref, z_ref = oracle_all_rows(w, q, k, v)
+    qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+    HW = w.HW
+    st = blin.BlockState(w.B, w.H, w.d)
+    sl = lambda a, f0, f1: a[:, :, f0 * HW:f1 * HW].contiguous()
+    blin.prefill(sl(qd, 0, 4), sl(kd, 0, 4), sl(vd, 0, 4), (4, w.Hg, w.Wg), w.F, w.split, w.theta, w.eps, state=st)
+    assert st.t_next == 4
+    S0, z0 = st.to_host()
+    # frames 4, 5, 6 would cross from block 1 into block 2
+    with pytest.raises(blin.BlinError, match="BLIN_ERR_SHAPE"):
+        blin.block_step(sl(qd, 4, 7), sl(kd, 4, 7), sl(vd, 4, 7), w.Hg, w.Wg, 3, w.split, st,
+                        theta=w.theta, eps=w.eps, block_frames=w.F)
+    S1, z1 = st.to_host()
+    assert st.t_next == 4 and torch.equal(S0, S1) and torch.equal(z0, z1)
+    o45 = blin.block_step(sl(qd, 4, 6), sl(kd, 4, 6), sl(vd, 4, 6), w.Hg, w.Wg, 2, w.split, st,
+                          theta=w.theta, eps=w.eps, block_frames=w.F)
+    o68 = blin.block_step(sl(qd, 6, 9), sl(kd, 6, 9), sl(vd, 6, 9), w.Hg, w.Wg, 3, w.split, st,
+                          theta=w.theta, eps=w.eps, block_frames=w.F)
+    torch.cuda.synchronize()
+    assert rel_err(host(o45).reshape(-1, 2 * HW, w.d), ref[:, 4 * HW:6 * HW]) <= TOL["bf16"]
+    assert rel_err(host(o68).reshape(-1, 3 * HW, w.d), ref[:, 6 * HW:]) <= TOL["bf16"]
+    assert st.t_next == 9
+    S, z = st.to_host()
+    assert rel_err(S.numpy().reshape(S_ref.shape), S_ref) <= 5e-3
+    assert rel_err(z.numpy().reshape(z_ref.shape), z_ref) <= 1e-5
