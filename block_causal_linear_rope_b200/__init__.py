@@ -21,7 +21,7 @@ from typing import Optional, Sequence, Tuple
 
 import torch
 
-__all__ = ["BlinError", "BlockState", "prefill", "block_step", "workspace_size", "device_status",
+__all__ = ["BlinError", "BlockState", "Layout", "prefill", "block_step", "workspace_size", "device_status",
            "last_path", "LaunchTimer", "KERNELS", "lib", "LIB_PATH", "F32", "BF16"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +31,10 @@ F32, BF16 = 0, 1
 _STATUS = {0: "BLIN_OK", -1: "BLIN_ERR_INVALID_ARG", -2: "BLIN_ERR_SHAPE", -3: "BLIN_ERR_DTYPE",
            -4: "BLIN_ERR_ALIGN", -5: "BLIN_ERR_WORKSPACE", -6: "BLIN_ERR_STATE", -7: "BLIN_ERR_CUDA",
            -8: "BLIN_ERR_DEVICE"}
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("token", ctypes.c_longlong), ("head", ctypes.c_longlong), ("batch", ctypes.c_longlong)]
 
 
 class BlinError(RuntimeError):
@@ -64,6 +68,11 @@ def _load() -> ctypes.CDLL:
     L.blin_prefill_workspace_size.restype = S
     L.blin_prefill.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), P, P, S, P]
     L.blin_block_step.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), P, I, P]
+    LP = ctypes.POINTER(Layout)
+    L.blin_prefill_strided.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), LP, LP, P, P, S, P]
+    L.blin_prefill_strided.restype = I
+    L.blin_block_step_strided.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(Geom), LP, LP, P, I, P]
+    L.blin_block_step_strided.restype = I
     L.blin_last_path.argtypes = []
     L.blin_last_path.restype = I
     L.blin_last_error.restype = ctypes.c_char_p
@@ -181,10 +190,20 @@ def _check_qkv(q, k, v):
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not isinstance(t, torch.Tensor) or not t.is_cuda:
             raise TypeError(f"{name} must be a CUDA tensor")
-        if t.dim() != 4 or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError(f"{name} must be a [B, H, N, d] tensor with d contiguous")
     if not (q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype):
         raise ValueError("q, k and v must share shape and dtype")
+    if not (q.stride() == k.stride() == v.stride()):
+        raise ValueError("q, k and v must share strides (one layout for the three)")
+
+
+def _layouts(q: torch.Tensor, out: torch.Tensor):
+    """(qkv layout, o layout) for the strided entry points, or None when all are contiguous."""
+    if q.is_contiguous() and out.is_contiguous():
+        return None
+    lay = lambda t: Layout(t.stride(2), t.stride(1), t.stride(0))
+    return lay(q), lay(out)
 
 
 def workspace_size(B: int, H: int, d: int, grid: Sequence[int], block_frames: int,
@@ -200,7 +219,12 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Sequence[in
             rope_split: Sequence[int], theta: float = 1e4, eps: float = 1e-6,
             state: Optional[BlockState] = None, out: Optional[torch.Tensor] = None,
             workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Block-causal linear attention over the frames grid=(T, Hg, Wg) (N = T*Hg*Wg)."""
+    """Block-causal linear attention over the frames grid=(T, Hg, Wg) (N = T*Hg*Wg).
+
+    q, k, v are [B, H, N, d] views with d contiguous; they may be strided (for
+    instance the q/k/v slices of a fused [B, N, 3, H, d] projection output, seen
+    as [B, H, N, d]) as long as the three share one layout.  `out` may be a
+    strided view too (default: a new contiguous tensor)."""
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
     T, Hg, Wg = (int(x) for x in grid)
@@ -208,15 +232,19 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Sequence[in
         raise ValueError(f"N={N} but T*Hg*Wg={T * Hg * Wg}")
     g = _geom(T, Hg, Wg, block_frames, rope_split, theta, eps)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
     need = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    _check(lib.blin_prefill(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-                            _dtype_code(q), B, H, d, ctypes.byref(g),
-                            state.handle if state is not None else None,
-                            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)))
+    args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+            ctypes.c_void_p(out.data_ptr()), _dtype_code(q), B, H, d, ctypes.byref(g))
+    tail = (state.handle if state is not None else None, ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+            _stream(stream))
+    lays = _layouts(q, out)
+    if lays is None:
+        _check(lib.blin_prefill(*args, *tail))
+    else:
+        _check(lib.blin_prefill_strided(*args, ctypes.byref(lays[0]), ctypes.byref(lays[1]), *tail))
     return out
 
 
@@ -226,18 +254,23 @@ def block_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Hg: int, Wg: i
                block_frames: Optional[int] = None) -> torch.Tensor:
     """One autoregressive block of `frames` latent frames read against (and, if
     commit, added to) the cached state.  `block_frames` is the causal block
-    length F (default: `frames`); the call's frames must lie in one block."""
+    length F (default: `frames`); the call's frames must lie in one block.
+    Strided views are accepted as for prefill()."""
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
     if N != frames * Hg * Wg:
         raise ValueError(f"N={N} but frames*Hg*Wg={frames * Hg * Wg}")
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
     g = _geom(frames, Hg, Wg, frames if block_frames is None else block_frames, rope_split, theta, eps)
-    _check(lib.blin_block_step(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                               ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-                               _dtype_code(q), B, H, d, ctypes.byref(g), state.handle,
-                               1 if commit else 0, _stream(stream)))
+    args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+            ctypes.c_void_p(out.data_ptr()), _dtype_code(q), B, H, d, ctypes.byref(g))
+    lays = _layouts(q, out)
+    if lays is None:
+        _check(lib.blin_block_step(*args, state.handle, 1 if commit else 0, _stream(stream)))
+    else:
+        _check(lib.blin_block_step_strided(*args, ctypes.byref(lays[0]), ctypes.byref(lays[1]), state.handle,
+                                           1 if commit else 0, _stream(stream)))
     return out
 
 
@@ -249,11 +282,14 @@ def last_path() -> str:
     return PATHS[int(lib.blin_last_path())]
 
 
+# Launch slots of one call, in order.  The tensor-core path launches three
+# kernels (partial states, block scan, output); the CUDA-core path also builds
+# a RoPE table first.
 KERNELS = ("rope_table", "partial_states", "block_scan", "output")
-# Algorithmic HBM bytes of each launch per token*head, in units of d * element size:
-# pass 1 reads K and V, pass 2 reads Q and writes O; the scan and the table move no
-# per-token bytes (None: not a roofline candidate).
-KERNEL_BYTES_PER_UNIT = {"rope_table": None, "partial_states": 2, "block_scan": None, "output": 2}
+# Algorithmic HBM bytes per token*head of each launch, in units of d * element
+# size: pass 1 reads K and V, pass 2 reads Q and writes O (the scan and the
+# table move no per-token bytes).
+KERNEL_BYTES_PER_UNIT = {"partial_states": 2, "output": 2}
 
 
 class LaunchTimer:

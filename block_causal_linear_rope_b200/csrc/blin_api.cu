@@ -52,23 +52,11 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------------- geometry
-// SMs of the current device (cached per device).
-static int device_sms() {
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
 struct Plan {
     KGeom g;
     int d;
-    size_t tab_bytes, part_bytes, prefix_bytes;
+    bool tc;  // tensor-core path
+    size_t ctl_bytes, tab_bytes, part_bytes, prefix_bytes;
 };
 
 static blin_status check_common(int B, int H, int d, int T, int Hg, int Wg, const int split[3],
@@ -89,18 +77,39 @@ static blin_status check_common(int B, int H, int d, int T, int Hg, int Wg, cons
     const long long HW = (long long)Hg * Wg;
     const long long N = (long long)T * HW;
     const long long rows = (long long)B * H * N;
-    if (HW > (1 << 30) || rows >= (1LL << 31) || rows * d >= (1LL << 40))
+    if (HW > (1 << 30) || N >= (1LL << 31) || rows >= (1LL << 40) || (long long)B * H >= (1LL << 24))
         return fail(BLIN_ERR_SHAPE, "problem too large (B*H*N = %lld rows)", rows);
     return BLIN_OK;
 }
 
-// Builds the call geometry; `one_block` treats the whole call as one block.
+// Tensor-core path, pass 1: state chunks per block, of about kChunkTiles32 /
+// kChunkTiles64 tiles, split evenly.  The count is a function of the block's
+// length and d only (never of the call, the number of heads or the device), so
+// a head's block reduces in the same chunks whether it arrives in a prefill, in
+// a block step or in a call with other heads.
+static constexpr int kChunkTiles32 = 5, kChunkTiles64 = 8;
+static int tc_chunks(long long L, int d) {
+    const long long nt = (L + kTile - 1) / kTile;
+    const long long ct = d == 32 ? kChunkTiles32 : kChunkTiles64;
+    return (int)std::max(1LL, (nt + ct - 1) / ct);
+}
+// Tensor-core path, pass 2: query groups of up to kGroupTiles tiles per block.
+static int tc_groups(long long L) {
+    const long long nt = (L + kTile - 1) / kTile;
+    return (int)std::max(1LL, (nt + kGroupTiles - 1) / kGroupTiles);
+}
+// CUDA-core path: 1024-token chunks.
+static int simt_chunks(long long L) { return (int)std::max(1LL, (L + kChunk - 1) / kChunk); }
+
+// Builds the call geometry; `one_block` treats the whole call as one block;
+// `for_size` sizes for the worst case over the starting frame (and both paths).
 static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0, bool one_block,
-                      const int split[3], float eps, bool for_size = false) {
+                      const int split[3], float eps, bool tc, bool for_size = false) {
     Plan p{};
     KGeom &g = p.g;
     p.d = d;
     g.BH = B * H;
+    g.H = H;
     g.T = T;
     g.Hg = Hg;
     g.Wg = Wg;
@@ -118,55 +127,67 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
         g.nblk = T > 0 ? 1 + (T - g.first_end + F - 1) / F : 0;
         if (for_size) g.nblk = (T + F - 1) / F + 1;  // worst case over t0
     }
-    const long long max_blk_tok = (long long)(one_block ? T : (F < T ? F : T)) * g.HW;
-    g.cpb = (int)((max_blk_tok + kChunk - 1) / kChunk);
-    if (g.cpb < 1) g.cpb = 1;
-    // Output groups of up to kQTiles query tiles; a call with few tiles (a decode
-    // block) uses smaller groups, so that every pipeline of the output kernel gets
-    // several (results do not depend on the grouping).
-    g.qgt = kQTiles;
-    if (!for_size) {
-        const long long tiles_per_blk = (max_blk_tok + kTile - 1) / kTile;
-        const long long pipelines = 2LL * device_sms();
-        while (g.qgt > 2 && (long long)g.BH * g.nblk * ((tiles_per_blk + g.qgt - 1) / g.qgt) < 4 * pipelines)
-            g.qgt /= 2;
-    }
-    const int qtok = g.qgt * kTile;
-    g.qcpb = (int)((max_blk_tok + qtok - 1) / qtok);
-    if (g.qcpb < 1) g.qcpb = 1;
     g.pt = split[0] / 2;
     g.py = split[1] / 2;
     g.px = split[2] / 2;
     g.eps = eps;
     g.tab_y = T * g.pt;
     g.tab_x = g.tab_y + Hg * g.py;
-    // chunks of one head: sum over blocks of ceil(block tokens / chunk)
-    long long chunks = 0;
-    for (int b = 0; b < g.nblk && !for_size; ++b)
-        chunks += ((long long)(block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
-    g.chunks_per_bh = (int)chunks;
-    // The tensor-core kernels keep the call's whole RoPE table in shared memory;
-    // a call whose table does not fit next to their rings takes the CUDA-core path.
+    // The tensor-core kernel keeps the call's whole RoPE table in shared memory;
+    // a call whose table does not fit next to its rings takes the CUDA-core path.
     const long long tab_entries = (long long)T * g.pt + (long long)Hg * g.py + (long long)Wg * g.px;
     g.tab_smem_bytes = (int)std::min<long long>(tab_entries * (long long)sizeof(float2), 1 << 30);
     g.tab_smem = g.tab_smem_bytes <= tc_table_smem_limit(d) ? 1 : 0;
+    tc = tc && g.tab_smem;
+    p.tc = tc;
+    // block lengths (tokens): the first, a middle and the last block
+    const long long HW = g.HW;
+    const long long Lf = (long long)g.first_end * HW, Lm = (long long)g.F * HW;
+    const long long Ll = g.nblk >= 2 ? (long long)(T - g.first_end - (g.nblk - 2) * g.F) * HW : Lf;
+    const long long Lmax = (long long)(one_block ? T : std::min(F, T)) * HW;
+    const int mids = g.nblk > 2 ? g.nblk - 2 : 0;
+    if (for_size) {
+        g.cpb = std::max(tc_chunks(Lmax, d), simt_chunks(Lmax));
+    } else {
+        auto chunks = [&](long long L) { return tc ? tc_chunks(L, d) : simt_chunks(L); };
+        g.nc_first = chunks(Lf);
+        g.nc_mid = chunks(Lm);
+        g.nc_last = chunks(Ll);
+        g.ng_first = tc_groups(Lf);
+        g.ng_mid = tc_groups(Lm);
+        g.ng_last = tc_groups(Ll);
+        g.U1 = g.nblk == 0 ? 0 : g.nc_first + mids * g.nc_mid + (g.nblk >= 2 ? g.nc_last : 0);
+        g.U2 = g.nblk == 0 ? 0 : g.ng_first + mids * g.ng_mid + (g.nblk >= 2 ? g.ng_last : 0);
+        g.cpb = std::max(g.nc_first, g.nblk >= 2 ? g.nc_last : 0);
+        if (mids > 0) g.cpb = std::max(g.cpb, g.nc_mid);
+    }
+    if (g.cpb < 1) g.cpb = 1;
     const size_t E = (size_t)d * d + d;
+    p.ctl_bytes = 256;  // work counters
     p.tab_bytes = align256(sizeof(float2) * ((size_t)T * g.pt + (size_t)Hg * g.py + (size_t)Wg * g.px + 1));
     p.part_bytes = align256(sizeof(float) * (size_t)g.BH * g.nblk * g.cpb * E);
     p.prefix_bytes = align256(sizeof(float) * (size_t)g.BH * g.nblk * E);
+    // contiguous [B][H][N][d] unless the caller says otherwise
+    g.lq = g.lo = Layout{d, (long long)g.N * d, (long long)H * g.N * d};
     return p;
 }
 
-// 256 bytes of alignment slack, 256 for the work counters, then the tables and states
-static size_t plan_bytes(const Plan &p) { return 512 + p.tab_bytes + p.part_bytes + p.prefix_bytes; }
+// 256 bytes of alignment slack, then the work counters, RoPE table, chunk partials, prefixes
+static size_t plan_bytes(const Plan &p) { return 256 + p.ctl_bytes + p.tab_bytes + p.part_bytes + p.prefix_bytes; }
 
 static void plan_bind(Plan &p, void *ws) {
     uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255);
-    p.g.sched = reinterpret_cast<unsigned int *>(base);
-    base += 256;
+    p.g.ctl = reinterpret_cast<unsigned int *>(base);
+    base += p.ctl_bytes;
     p.g.tab = reinterpret_cast<const float2 *>(base);
     p.g.part = reinterpret_cast<float *>(base + p.tab_bytes);
     p.g.prefix = reinterpret_cast<float *>(base + p.tab_bytes + p.part_bytes);
+}
+
+// Bytes of a prefill workspace for this shape (both paths, any starting frame).
+static size_t prefill_bytes(int B, int H, int d, const blin_geom *g) {
+    Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, 0, false, g->rope_split, g->eps, false, true);
+    return plan_bytes(p);
 }
 
 // ---------------------------------------------------------------- contexts
@@ -217,18 +238,24 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2D map over [rows][d] bf16 rows, 128-row boxes, swizzle = row width (64 B / 128 B).
-// 2D view [rows][d] bf16 with `box_rows`-row boxes, swizzled to the row size.
-static bool make_map(CUtensorMap *m, const void *base, long long rows, int d, int box_rows = kTile) {
+// 4D view of a bf16 [B][H][N][d] operand with element strides `l`: dimensions
+// (feature, then token and head ordered by stride, then batch), `box_rows`
+// tokens per box, swizzled to the row size (64 B at d = 32, 128 B at d = 64).
+// *swap = 1 when the head dimension comes before the token one.  Tokens past
+// N read as zeros.
+static bool make_map4(CUtensorMap *m, const void *base, const Layout &l, int B, int H, int N, int d, int box_rows,
+                      int *swap) {
     EncodeTiledFn enc = encode_fn();
     if (enc == nullptr) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+    const bool sw = l.head < l.tok;
+    *swap = sw ? 1 : 0;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)(sw ? H : N), (cuuint64_t)(sw ? N : H), (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)(sw ? l.head : l.tok) * 2, (cuuint64_t)(sw ? l.tok : l.head) * 2,
+                             (cuuint64_t)l.batch * 2};
+    cuuint32_t box[4] = {(cuuint32_t)d, (cuuint32_t)(sw ? 1 : box_rows), (cuuint32_t)(sw ? box_rows : 1), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -243,40 +270,51 @@ static void mark(int i, bool after, cudaStream_t s) {
     if (g_timing != nullptr) cudaEventRecord(g_timing[2 * i + (after ? 1 : 0)], s);
 }
 
+// Enqueues the call.
 static blin_status run(Plan &p, const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                        const float *S_in, const float *z_in, float *S_out, float *z_out, double theta,
-                       const int split[3], cudaStream_t s) {
+                       cudaStream_t s) {
     p.g.S_in = S_in;
     p.g.z_in = z_in;
     p.g.theta = theta;
     p.g.S_out = S_out;
     p.g.z_out = z_out;
-    const KGeom &g = p.g;
+    KGeom &g = p.g;
     const int d = p.d;
-    const bool tc = dt == BLIN_BF16 && tc_supported(d, split) && g.tab_smem;
+    const bool tc = p.tc;
     g_last_path = tc ? BLIN_PATH_TENSOR_CORE : BLIN_PATH_CUDA_CORE;
-    CUtensorMap mq, mk, mv, mo;
+    cudaError_t e;
     if (tc) {
-        const long long rows = (long long)g.BH * g.N;
-        if (!make_map(&mq, q, rows, d) || !make_map(&mk, k, rows, d) || !make_map(&mv, v, rows, d) ||
-            !make_map(&mo, o, rows, d, 32))
-            return fail(BLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
+        CUtensorMap mq, mk, mv;
+        int sk = 0, sv = 0;
+        const int B = g.BH / g.H;
+        if (!make_map4(&mq, q, g.lq, B, g.H, g.N, d, kTile, &g.swap_q) ||
+            !make_map4(&mk, k, g.lq, B, g.H, g.N, d, kTile, &sk) || !make_map4(&mv, v, g.lq, B, g.H, g.N, d, kTile, &sv))
+            return fail(BLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or strides rejected)");
+        // both kernels hand out their work through counters that start at zero
+        if ((e = cudaMemsetAsync(g.ctl, 0, 4 * sizeof(unsigned int), s)) != cudaSuccess)
+            return cuda_fail(e, "work counter reset");
+        mark(1, false, s);
+        if ((e = launch_partial_tc(g, d, mk, mv, s)) != cudaSuccess) return cuda_fail(e, "partial-state launch");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        mark(1, true, s);
+        mark(2, false, s);
+        if ((e = launch_scan(g, d, S_in, z_in, S_out, z_out, s)) != cudaSuccess) return cuda_fail(e, "scan launch");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        mark(2, true, s);
+        mark(3, false, s);
+        if ((e = launch_output_tc(g, d, mq, o, s)) != cudaSuccess) return cuda_fail(e, "output launch");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        mark(3, true, s);
+        return BLIN_OK;
     }
     const bool bf = dt == BLIN_BF16;
-    cudaError_t e;
     mark(0, false, s);
-    // the tensor-core kernels build their RoPE tables in shared memory themselves
-    if (!tc) {
-        if ((e = launch_rope_table(g, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-    }
+    if ((e = launch_rope_table(g, s)) != cudaSuccess) return cuda_fail(e, "rope table launch");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(0, true, s);
-    // the tensor-core passes hand out work units through counters that start at zero
-    if (tc && (e = cudaMemsetAsync(g.sched, 0, 4 * sizeof(unsigned int), s)) != cudaSuccess)
-        return cuda_fail(e, "work counter reset");
     mark(1, false, s);
-    e = tc ? launch_partial_tc(g, d, mk, mv, s) : launch_partial_simt(g, d, bf, k, v, s);
-    if (e != cudaSuccess) return cuda_fail(e, "partial-state launch");
+    if ((e = launch_partial_simt(g, d, bf, k, v, s)) != cudaSuccess) return cuda_fail(e, "partial-state launch");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(1, true, s);
     mark(2, false, s);
@@ -284,8 +322,7 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
     g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(2, true, s);
     mark(3, false, s);
-    e = tc ? launch_output_tc(g, d, mq, mo, o, s) : launch_output_simt(g, d, bf, q, o, s);
-    if (e != cudaSuccess) return cuda_fail(e, "output launch");
+    if ((e = launch_output_simt(g, d, bf, q, o, s)) != cudaSuccess) return cuda_fail(e, "output launch");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     mark(3, true, s);
     return BLIN_OK;
@@ -438,14 +475,41 @@ blin_status blin_state_copy_from_host(blin_state *st, const void *host, size_t b
     return BLIN_OK;
 }
 
+// Grows the state's block-step scratch to `need` bytes.
 static blin_status ensure_scratch(blin_state *st, size_t need, cudaStream_t s) {
     if (st->scratch_bytes >= need) return BLIN_OK;
     void *p = nullptr;
     cudaError_t e = cudaMallocAsync(&p, need, s);
-    if (e != cudaSuccess) return cuda_fail(e, "block-step scratch allocation");
+    if (e != cudaSuccess) {
+        if (p) cudaFreeAsync(p, s);
+        return cuda_fail(e, "block-step scratch allocation");
+    }
     if (st->scratch) cudaFreeAsync(st->scratch, s);
     st->scratch = p;
     st->scratch_bytes = need;
+    return BLIN_OK;
+}
+
+// Element strides of q/k/v (or o) from the caller's layout (NULL: contiguous).
+static blin_status get_layout(const blin_layout *l, int B, int H, int N, int d, blin_dtype dt, const char *name,
+                              Layout *out) {
+    if (l == nullptr) {
+        *out = Layout{d, (long long)N * d, (long long)H * N * d};
+        return BLIN_OK;
+    }
+    Layout x{l->token, l->head, l->batch};
+    // a dimension of extent 1 never moves: give it a harmless stride
+    if (H == 1) x.head = x.tok * (long long)std::max(N, 1);
+    if (B == 1) x.batch = std::max(x.tok * (long long)std::max(N, 1), x.head * (long long)H);
+    if (x.tok < d || x.head < d || x.batch < d)
+        return fail(BLIN_ERR_SHAPE, "%s strides (token %lld, head %lld, batch %lld) must each be >= d = %d", name,
+                    l->token, l->head, l->batch, d);
+    const long long es = dt == BLIN_BF16 ? 2 : 4;
+    if ((x.tok * es) % 16 || (x.head * es) % 16 || (x.batch * es) % 16)
+        return fail(BLIN_ERR_ALIGN, "%s strides must be multiples of 16 bytes", name);
+    if (x.tok * es >= (1LL << 40) || x.head * es >= (1LL << 40) || x.batch * es >= (1LL << 40))
+        return fail(BLIN_ERR_SHAPE, "%s strides too large", name);
+    *out = x;
     return BLIN_OK;
 }
 
@@ -456,7 +520,7 @@ blin_status blin_state_reserve(blin_state *st, long max_block_tokens, blin_strea
         return fail(BLIN_ERR_INVALID_ARG, "max_block_tokens out of range");
     // Widest table: all tokens on one axis of one frame (Hgt = 1, Wid = tokens).
     const int split_wide[3] = {0, 0, st->d};
-    Plan p = make_plan(st->B, st->H, st->d, 1, 1, (int)max_block_tokens, 1, 0, true, split_wide, 0.f);
+    Plan p = make_plan(st->B, st->H, st->d, 1, 1, (int)max_block_tokens, 1, 0, true, split_wide, 0.f, false, true);
     return ensure_scratch(st, plan_bytes(p), static_cast<cudaStream_t>(stream));
 }
 
@@ -464,18 +528,21 @@ size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom *g) {
     if (g == nullptr) return 0;
     if (check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps) != BLIN_OK) return 0;
     if (g->block_frames < 1) return 0;
-    Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, 0, false, g->rope_split, g->eps, true);
-    return plan_bytes(p);
+    return prefill_bytes(B, H, d, g);
 }
 
-blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
-                         int H, int d, const blin_geom *g, blin_state *st, void *workspace,
-                         size_t ws_bytes, blin_stream stream) {
+static blin_status prefill_impl(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B, int H,
+                                int d, const blin_geom *g, const blin_layout *lqkv, const blin_layout *lout,
+                                blin_state *st, void *workspace, size_t ws_bytes, blin_stream stream) {
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;
     if (g->block_frames < 1) return fail(BLIN_ERR_INVALID_ARG, "block_frames must be >= 1");
     if ((rc = check_io(q, k, v, o, dt)) != BLIN_OK) return rc;
+    const int N = g->T * g->Hgt * g->Wid;
+    Layout lq, lo;
+    if ((rc = get_layout(lqkv, B, H, N, d, dt, "q/k/v", &lq)) != BLIN_OK) return rc;
+    if ((rc = get_layout(lout, B, H, N, d, dt, "o", &lo)) != BLIN_OK) return rc;
     if (st != nullptr) {
         if ((rc = check_state(st)) != BLIN_OK) return rc;
         if (st->B != B || st->H != H || st->d != d)
@@ -483,16 +550,19 @@ blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, b
                         st->d, B, H, d);
     }
     if (g->T == 0) return BLIN_OK;
-    const size_t need = blin_prefill_workspace_size(B, H, d, g);
+    const size_t need = prefill_bytes(B, H, d, g);
     if (workspace == nullptr || ws_bytes < need)
         return fail(BLIN_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? ws_bytes : 0, need);
     if (!aligned16(workspace)) return fail(BLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
     const int t0 = st ? st->t_next : 0;
     if ((long long)t0 + g->T >= (1LL << 30)) return fail(BLIN_ERR_SHAPE, "frame index overflow");
-    Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, t0, false, g->rope_split, g->eps);
+    const bool tc = dt == BLIN_BF16 && tc_supported(d, g->rope_split);
+    Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, t0, false, g->rope_split, g->eps, tc);
+    p.g.lq = lq;
+    p.g.lo = lo;
     plan_bind(p, workspace);
     rc = run(p, q, k, v, o, dt, st ? st->S : nullptr, st ? st->z : nullptr, st ? st->S : nullptr,
-             st ? st->z : nullptr, (double)g->theta, g->rope_split, static_cast<cudaStream_t>(stream));
+             st ? st->z : nullptr, (double)g->theta, static_cast<cudaStream_t>(stream));
     if (rc != BLIN_OK) return rc;
     if (st) {
         if ((rc = mark_state_use(st, static_cast<cudaStream_t>(stream))) != BLIN_OK) return rc;
@@ -501,8 +571,9 @@ blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, b
     return BLIN_OK;
 }
 
-blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
-                            int H, int d, const blin_geom *g, blin_state *st, int commit, blin_stream stream) {
+static blin_status block_step_impl(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
+                                   int H, int d, const blin_geom *g, const blin_layout *lqkv,
+                                   const blin_layout *lout, blin_state *st, int commit, blin_stream stream) {
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;
@@ -511,6 +582,10 @@ blin_status blin_block_step(const void *q, const void *k, const void *v, void *o
     if (F < 1) return fail(BLIN_ERR_INVALID_ARG, "block_frames must be >= 1");
     if (commit != 0 && commit != 1) return fail(BLIN_ERR_INVALID_ARG, "commit must be 0 or 1");
     if ((rc = check_io(q, k, v, o, dt)) != BLIN_OK) return rc;
+    const int N = frames * g->Hgt * g->Wid;
+    Layout lq, lo;
+    if ((rc = get_layout(lqkv, B, H, N, d, dt, "q/k/v", &lq)) != BLIN_OK) return rc;
+    if ((rc = get_layout(lout, B, H, N, d, dt, "o", &lo)) != BLIN_OK) return rc;
     if ((rc = check_state(st)) != BLIN_OK) return rc;
     if (st->B != B || st->H != H || st->d != d)
         return fail(BLIN_ERR_STATE, "state is B=%d H=%d d=%d, call is B=%d H=%d d=%d", st->B, st->H, st->d,
@@ -522,15 +597,41 @@ blin_status blin_block_step(const void *q, const void *k, const void *v, void *o
                     "frames [%d, %d) cross a block boundary (block_frames %d): a block step covers one block",
                     st->t_next, st->t_next + frames, F);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    Plan p = make_plan(B, H, d, frames, g->Hgt, g->Wid, frames, st->t_next, true, g->rope_split, g->eps);
+    const bool tc = dt == BLIN_BF16 && tc_supported(d, g->rope_split);
+    Plan p = make_plan(B, H, d, frames, g->Hgt, g->Wid, frames, st->t_next, true, g->rope_split, g->eps, tc);
+    p.g.lq = lq;
+    p.g.lo = lo;
     if ((rc = ensure_scratch(st, plan_bytes(p), s)) != BLIN_OK) return rc;
     plan_bind(p, st->scratch);
     rc = run(p, q, k, v, o, dt, st->S, st->z, commit ? st->S : nullptr, commit ? st->z : nullptr,
-             (double)g->theta, g->rope_split, s);
+             (double)g->theta, s);
     if (rc != BLIN_OK) return rc;
     if ((rc = mark_state_use(st, s)) != BLIN_OK) return rc;
     if (commit) st->t_next += frames;
     return BLIN_OK;
+}
+
+blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B, int H, int d,
+                         const blin_geom *g, blin_state *st, void *workspace, size_t ws_bytes, blin_stream stream) {
+    return prefill_impl(q, k, v, o, dt, B, H, d, g, nullptr, nullptr, st, workspace, ws_bytes, stream);
+}
+
+blin_status blin_prefill_strided(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B, int H,
+                                 int d, const blin_geom *g, const blin_layout *qkv_layout,
+                                 const blin_layout *o_layout, blin_state *st, void *workspace, size_t ws_bytes,
+                                 blin_stream stream) {
+    return prefill_impl(q, k, v, o, dt, B, H, d, g, qkv_layout, o_layout, st, workspace, ws_bytes, stream);
+}
+
+blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B, int H,
+                            int d, const blin_geom *g, blin_state *st, int commit, blin_stream stream) {
+    return block_step_impl(q, k, v, o, dt, B, H, d, g, nullptr, nullptr, st, commit, stream);
+}
+
+blin_status blin_block_step_strided(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
+                                    int H, int d, const blin_geom *g, const blin_layout *qkv_layout,
+                                    const blin_layout *o_layout, blin_state *st, int commit, blin_stream stream) {
+    return block_step_impl(q, k, v, o, dt, B, H, d, g, qkv_layout, o_layout, st, commit, stream);
 }
 
 int blin_last_path(void) { return g_last_path; }

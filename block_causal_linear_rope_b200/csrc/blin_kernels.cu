@@ -118,15 +118,13 @@ static cudaError_t set_smem(int bytes) {
 // Largest RoPE table (bytes) the tensor-core kernels can hold in shared memory
 // next to their rings (227 KB per CTA).
 int tc_table_smem_limit(int d) {
-    const int fixed = d == 32 ? std::max(P1<32>::FIXED, P2<32>::FIXED) : std::max(P1<64>::FIXED, P2<64>::FIXED);
+    const int fixed = d == 32 ? std::max(K1Cfg<32>::FIXED, K2Cfg<32>::FIXED) : std::max(K1Cfg<64>::FIXED, K2Cfg<64>::FIXED);
     return std::min(24 * 1024, 227 * 1024 - fixed);
 }
 
-// Launch with programmatic dependent launch allowed: the kernel may start
-// while the previous kernel in the stream finishes; it calls
-// griddepcontrol.wait before reading anything that kernel wrote.
-// `pdl` false gives an ordinary launch (the first kernel of a call, which reads
-// the caller's inputs, always waits for everything before it).
+// Launch with programmatic dependent launch allowed when `pdl`: the kernel may
+// start while the previous kernel in the stream finishes; it calls
+// griddepcontrol.wait before reading what that kernel wrote.
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_ex(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
                              Args &&...args) {
@@ -142,75 +140,59 @@ static cudaError_t launch_ex(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3
     cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
-                              Args &&...args) {
-    return launch_ex(true, kernel, grid, block, smem, s, std::forward<Args>(args)...);
-}
 
 cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
                         float *z_out, cudaStream_t s) {
     const long long cols = (long long)g.BH * ((d * d + d) / 4);  // (head, float4 column) pairs: one thread each
     const dim3 grid((unsigned)((cols + 255) / 256));
-    cudaError_t e = launch_pdl(scan_kernel, grid, dim3(256), 0, s, g, d, S_in, z_in, S_out, z_out);
+    cudaError_t e = launch_ex(true, scan_kernel, grid, dim3(256), 0, s, g, d, S_in, z_in, S_out, z_out);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-// Persistent grid: as many CTAs as fit on the device at once, never more than
-// there are work units.
-template <auto Kernel>
-static int persistent_grid(int smem, int threads, long long units) {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 1;
-    }
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, Kernel, threads, smem) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    const long long n = (long long)sms * per_sm;
-    return (int)(units < n ? (units > 0 ? units : 1) : n);
+// SMs of the current device (the persistent grid: one CTA per SM).
+static int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+        n = 148;
+    return n;
 }
 
+// Persistent launch: one CTA per SM, never more CTAs than pipelines have units.
 template <auto Kernel, typename... Args>
-static cudaError_t launch_persistent(bool pdl, int smem, int threads, long long units, cudaStream_t s,
+static cudaError_t launch_persistent(bool pdl, int smem, int threads, long long pipes_needed, int np, cudaStream_t s,
                                      Args &&...args) {
     cudaError_t e = set_smem<Kernel>(smem);
     if (e != cudaSuccess) return e;
-    const int grid = persistent_grid<Kernel>(smem, threads, units);
+    const long long ctas = std::max(1LL, (pipes_needed + np - 1) / np);
+    const int grid = (int)std::min<long long>(device_sm_count(), ctas);
     e = launch_ex(pdl, Kernel, dim3(grid), dim3(threads), smem, s, std::forward<Args>(args)...);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv,
-                              cudaStream_t s) {
+cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv, cudaStream_t s) {
     int *wd = watchdog_ptr();
     if (wd == nullptr) return cudaErrorInvalidDevice;
-    const long long units = (long long)g.cpb * g.nblk * g.BH;
     const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
-    // a CTA runs NP pipelines, each taking every NP-th of the CTA's chunks
+    const long long units = (long long)g.BH * g.U1;
     if (d == 32)
-        return launch_persistent<partial_tc_kernel<32, 4, 6, 6>>(false, P1<32>::FIXED + tab, P1<32>::THREADS,
-                                                                 (units + P1<32>::NP - 1) / P1<32>::NP, s, mk, mv, g, wd);
-    return launch_persistent<partial_tc_kernel<64, 8, 12, 12>>(false, P1<64>::FIXED + tab, P1<64>::THREADS,
-                                                               (units + P1<64>::NP - 1) / P1<64>::NP, s, mk, mv, g, wd);
+        return launch_persistent<partial_tc_kernel<32, 4, 6, 6>>(false, K1Cfg<32>::FIXED + tab, K1Cfg<32>::THREADS, units,
+                                                                 K1Cfg<32>::NP, s, mk, mv, g, wd);
+    return launch_persistent<partial_tc_kernel<64, 8, 12, 12>>(false, K1Cfg<64>::FIXED + tab, K1Cfg<64>::THREADS, units,
+                                                               K1Cfg<64>::NP, s, mk, mv, g, wd);
 }
 
-cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, const CUtensorMap &mo, void *o,
-                             cudaStream_t s) {
+cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, void *o, cudaStream_t s) {
     int *wd = watchdog_ptr();
     if (wd == nullptr) return cudaErrorInvalidDevice;
-    const long long units = (long long)g.qcpb * g.nblk * g.BH;
     const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
+    const long long units = (long long)g.BH * g.U2;
     __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
-    // a CTA runs NP pipelines, each taking every NP-th of the CTA's groups
     if (d == 32)
-        return launch_persistent<output_tc_kernel<32, 4, 6, 6>>(true, P2<32>::FIXED + tab, P2<32>::THREADS,
-                                                                (units + P2<32>::NP - 1) / P2<32>::NP, s, mq, mo, g, ob, wd);
-    return launch_persistent<output_tc_kernel<64, 8, 12, 12>>(true, P2<64>::FIXED + tab, P2<64>::THREADS,
-                                                              (units + P2<64>::NP - 1) / P2<64>::NP, s, mq, mo, g, ob, wd);
+        return launch_persistent<output_tc_kernel<32, 4, 6, 6>>(true, K2Cfg<32>::FIXED + tab, K2Cfg<32>::THREADS, units,
+                                                                K2Cfg<32>::NP, s, mq, g, ob, wd);
+    return launch_persistent<output_tc_kernel<64, 8, 12, 12>>(true, K2Cfg<64>::FIXED + tab, K2Cfg<64>::THREADS, units,
+                                                              K2Cfg<64>::NP, s, mq, g, ob, wd);
 }
 
 }  // namespace blin

@@ -74,9 +74,7 @@ __global__ void __launch_bounds__(256) scan_kernel(KGeom g, int d, const float *
     const int bh = (int)(f / E4), e4 = (int)(f - (long long)bh * E4);
     const float4 *part = reinterpret_cast<const float4 *>(g.part) + (size_t)bh * g.nblk * g.cpb * E4 + e4;
     float4 *prefix = reinterpret_cast<float4 *>(g.prefix) + (size_t)bh * g.nblk * E4 + e4;
-    auto nchunks = [&](int b) {
-        return ((block_frame_end(g, b) - block_frame_begin(g, b)) * g.HW + kChunk - 1) / kChunk;
-    };
+    auto nchunks = [&](int b) { return units_of_block(g, b, g.nc_first, g.nc_mid, g.nc_last); };
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (S_in != nullptr)
         acc = 4 * e4 < d * d ? reinterpret_cast<const float4 *>(S_in + (size_t)bh * d * d)[e4]
@@ -128,6 +126,12 @@ __device__ __forceinline__ void store_val(__nv_bfloat16 *p, size_t i, float x) {
     p[i] = __float2bfloat16_rn(x);
 }
 
+// Element offset of token `tok` of head `bh` (= b * H + h) in a strided operand.
+__device__ __forceinline__ size_t row_off(const Layout &l, int H, int bh, int tok) {
+    const int b = bh / H, h = bh - b * H;
+    return (size_t)b * l.batch + (size_t)h * l.head + (size_t)tok * l.tok;
+}
+
 // (cos, sin) of RoPE pair p (0 <= p < d/2) at relative frame t, row y, column x.
 __device__ __forceinline__ float2 rope_cs(const KGeom &g, int p, int t, int y, int x) {
     if (p < g.pt) return g.tab[t * g.pt + p];
@@ -162,7 +166,7 @@ __global__ void __launch_bounds__(256) partial_simt_kernel(KGeom g, const Tin *k
             float a = 0.f, bb = 0.f, ra = 0.f, rb = 0.f, va = 0.f, vb = 0.f;
             if (r < n) {
                 const int tok = tok0 + t + r;
-                const size_t off = ((size_t)bh * g.N + tok) * D + 2 * p;
+                const size_t off = row_off(g.lq, g.H, bh, tok) + 2 * p;
                 a = fmaxf(load_val(k, off), 0.f);
                 bb = fmaxf(load_val(k, off + 1), 0.f);
                 va = load_val(v, off);
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(128) output_simt_kernel(KGeom g, const Tin *q,
     const int r = ts + threadIdx.x;
     if (r >= ntok) return;
     const int tok = tok0 + r;
-    const size_t off = ((size_t)bh * g.N + tok) * D;
+    const size_t off = row_off(g.lq, g.H, bh, tok), ooff = row_off(g.lo, g.H, bh, tok);
     const int tt = tok / g.HW, rem = tok - tt * g.HW, y = rem / g.Wg, x = rem - y * g.Wg;
     float rq[D];
     float den = 0.f;
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(128) output_simt_kernel(KGeom g, const Tin *q,
         float s = 0.f;
 #pragma unroll
         for (int i = 0; i < D; ++i) s = fmaf(rq[i], S[i][j], s);
-        store_val(o, off + j, s / den);
+        store_val(o, ooff + j, s / den);
     }
 }
 

@@ -1,21 +1,21 @@
-// Tensor-core path for bf16 Q/K/V on sm_100a (d = 32 or 64).
+// Tensor-core path for bf16 Q/K/V on sm_100a (d = 32 or 64): two persistent
+// warp-specialized kernels around the fixed-order block scan.
 //
-// Pass 1, partial_tc_kernel: per chunk (<= 1024 tokens of one block of one
-//   head) the partial states P = sum (R_m phi(k_m)) v_m^T and zp = sum phi(k_m)
-//   from one contraction
+// Pass 1, partial_tc_kernel: per state chunk (whole 128-token tiles of one
+//   block of one head) the partial states P = sum (R_m phi(k_m)) v_m^T and
+//   zp = sum phi(k_m) from one contraction
 //       [K~^T ; phi(K)^T] x [V | 1]      (tcgen05.mma, fp32 in TMEM)
 //   whose operands are MN-major views of the token-major tiles.
-// Pass 2, output_tc_kernel: per group of <= 8 query tiles of one block of one
-//   head, numerator and denominator from one contraction
+// Pass 2, output_tc_kernel: per group of query tiles of one block of one head,
+//   numerator and denominator from one contraction
 //       [Q~ | phi(Q)] x [[S, 0], [0, z_hi z_lo]] = [num | phi(q).z_hi | phi(q).z_lo]
 //   then o = num / (phi(q).z + eps) in fp32, stored as bf16.
 //
-// Both kernels are persistent (one CTA per SM) and split into roles (TMA
-// producer, transform warps, one MMA-issuing thread, epilogue) that hand tiles
-// to each other through mbarrier rings only; each CTA runs two such pipelines
-// at d = 32 (see the pass 1 comment for why).  Every wait is bounded
-// (ptx::mbar_wait_bounded), and work is ordered chunk-index major so the
-// short last chunks of every block run last.
+// Each CTA (one per SM) runs two pipelines at d = 32, one at d = 64.  A
+// pipeline is split into roles -- a TMA producer, four transform warps, one
+// MMA-issuing thread, four epilogue warps -- that hand tiles to each other
+// through mbarrier rings, and takes its work units one at a time from a
+// counter shared by the whole grid.  Every wait is bounded.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -239,293 +239,319 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
     if (lane == 0) ptx::mbar_arrive(bar);
 }
 
-// ============================================================================ pass 1
+// ============================================================================ work units
+// Unit r of a head (pass-1 chunks or pass-2 query groups, ordered by block):
+// block b and index c inside the block.
+__device__ __forceinline__ void unit_block(const KGeom &g, int r, int nf, int nm, int nl, int &b, int &c) {
+    if (r < nf) {
+        b = 0;
+        c = r;
+        return;
+    }
+    r -= nf;
+    const int mids = g.nblk > 2 ? g.nblk - 2 : 0;
+    if (r < mids * nm) {
+        b = 1 + r / nm;
+        c = r - (b - 1) * nm;
+        return;
+    }
+    b = g.nblk - 1;
+    c = r - mids * nm;
+}
+
+// 4D tensor-map coordinates (feature, token, head, batch) in the map's own
+// dimension order: dims 1 and 2 are ordered by stride, so `swap` puts the head
+// before the token (a token-interleaved [B][N][H][d] layout).
+struct MapCoord {
+    int y, z;
+};
+__device__ __forceinline__ MapCoord map_coord(int n, int h, int swap) { return swap ? MapCoord{h, n} : MapCoord{n, h}; }
+
+// ============================================================================ configuration
 template <int D>
-struct P1 {
+struct TcCfg {
     static constexpr int ROWB = 2 * D;
-    static constexpr int TB = kTile * ROWB;
-    static constexpr int M = D == 32 ? 64 : 128;          // [K~^T ; phi(K)^T]
-    static constexpr int N = D == 32 ? D + 8 : D + 16;   // [V | ones]
-    static constexpr int NP = D == 32 ? 2 : 1;           // independent pipelines per CTA (MMA issuers)
-    static constexpr int NK = D == 32 ? 4 : 3;           // K landing slots per pipeline (free once read)
-    static constexpr int NV = D == 32 ? 5 : 4;           // V landing slots per pipeline (free once the MMA is done)
-    static constexpr int NO = 2;                         // operand sets per pipeline: K~ | phi
-    static constexpr int NACC = 2;                       // TMEM accumulators per pipeline (chunks in flight)
-    static constexpr int ACOLS = D == 32 ? 64 : 128;     // TMEM columns per accumulator
-    static constexpr uint32_t TCOLS = NP * NACC * ACOLS;
-    static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
-    static constexpr int NBAR = 2 * NK + NV + NO + 2 * NACC;  // mbarriers per pipeline
-    static constexpr int CTRL = 1024;
-    static constexpr int BARS = 512;                     // mbarrier area at the start of the control block
-    static constexpr int RINGS = NP * (2 * NO + NK + NV) * TB;  // operand, K and V rings of all pipelines
-    static constexpr int FIXED = RINGS + TB + CTRL + 1024;  // + RoPE table
-    static constexpr int THREADS = 32 * 6 * NP;  // warps [0, 4NP) transform, then NP producers, NP MMA issuers
-    static_assert(NP * (NBAR + 1) * 8 <= BARS, "mbarriers (+ one drain barrier per pipeline) overflow their area");
-    static_assert(BARS + 4 * NP * (4 * NK + 4 * NO) + 16 <= CTRL, "control block overflow");
-    static_assert(NV > NO, "an operand slot's release is read from the V ring's tile-done barriers");
-    // the B operand's second N atom (the ones block) sits above every V slot
-    static_assert(NP * NV * TB < (1 << 18), "LBO field range");
-    static_assert(TCOLS <= 512, "TMEM holds 512 columns");
+    static constexpr int TB = kTile * ROWB;           // one 128-token tile: 8 KB (d = 32) / 16 KB (d = 64)
+    static constexpr int NP = D == 32 ? 2 : 1;        // pipelines per CTA
+    static constexpr int PIPE_WARPS = 10;             // per pipeline: 4 transform, 4 epilogue, producer, MMA
+    static constexpr int THREADS = 32 * PIPE_WARPS * NP;
+    static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;  // smem descriptor swizzle: 64B / 128B
+    static constexpr int ACOLS = D == 32 ? 64 : 128;       // TMEM columns per accumulator
+    static constexpr int NINFO = 16;                        // producer -> epilogue record ring
+    static constexpr int NO = 2;                            // operand slots
+    static constexpr int NA = 4;                            // TMEM accumulators per pipeline
+    static constexpr uint32_t TCOLS = 512;
+    static constexpr int E = D * D + D, E4 = E / 4;
+    // control block: [NP][BARS_PER_PIPE] mbarriers, 16 B of flags, [NP][INFO_PER_PIPE] record ints
+    static constexpr int BARS_PER_PIPE = 64;
+    static constexpr int INFO_PER_PIPE = 128;
+    static constexpr int OFF_FLAGS = NP * BARS_PER_PIPE * 8;
+    static constexpr int OFF_INFO = OFF_FLAGS + 16;
+    static constexpr int CTRL = (OFF_INFO + NP * INFO_PER_PIPE * 4 + 1023) / 1024 * 1024;
+    static_assert(NP * NA * ACOLS <= (int)TCOLS, "TMEM columns");
 };
 
-// Persistent, one CTA per SM (a kernel that uses tcgen05 gets one CTA per SM).
-// The CTA runs NP independent pipelines, so that NP threads issue MMAs: one
-// thread issues a tcgen05.mma about every 50 cycles and the eight M = 64 MMAs
-// a 128-token tile needs from one thread would not keep up with HBM, while two
-// issuers' MMAs overlap in the tensor core.  Chunks are taken in
-// chunk-index-major order (the short last chunk of every block comes last):
-// pipeline p of CTA j first takes chunk j + p * grid, then the next unclaimed
-// chunk from a work counter, so all pipelines finish within about one chunk.
-// Per pipeline: a producer thread lands each K tile and V tile with TMA in
-// two rings; four transform warps read K (its slot is free again at once) and
-// write the A operand (K~, phi(K)) into an operand ring; an MMA thread
-// accumulates [K~^T; phi^T] x [V | 1] into a TMEM accumulator per chunk,
-// taking V straight from its landing slot, and commits once per tile to that V
-// slot's tile-done barrier, which frees both the V slot and the tile's operand
-// slot.  Two tiles into the next chunk, the transform warps read the finished
-// accumulator back (each warp its TMEM subpartition) and write the chunk
-// partial to global memory.
+template <int D>
+struct K1Cfg : TcCfg<D> {
+    using B = TcCfg<D>;
+    static constexpr int M1 = D == 32 ? 64 : 128;          // [K~^T ; phi(K)^T]
+    static constexpr int N1 = D == 32 ? D + 8 : D + 16;    // [V | ones]
+    static constexpr int NK = D == 32 ? 4 : 3;             // K landing slots (free once read)
+    static constexpr int NV = 4;                           // V landing slots (free once the MMA is done)
+    static constexpr int PIPE = (NK + NV + 2 * B::NO) * B::TB;
+    static constexpr int OFF_ONES = B::NP * PIPE;          // above every V slot: positive LBO
+    static constexpr int OFF_CTRL = OFF_ONES + B::TB;
+    static constexpr int FIXED = OFF_CTRL + B::CTRL + 1024;  // + alignment slack; the RoPE table follows
+    static constexpr int NBAR = 2 * NK + NV + B::NO + 2 * B::NA + 2 * B::NINFO + 1;
+    static constexpr int NINF = 5 * NK + 4 * B::NO + B::NINFO;
+    static_assert(NBAR <= B::BARS_PER_PIPE && NINF <= B::INFO_PER_PIPE, "control block");
+    static_assert(NV > B::NO, "an operand slot's release is read from the V ring's tile-done barriers");
+    static_assert(OFF_ONES < (1 << 18), "LBO field range");
+    static_assert(PIPE % 1024 == 0, "pipelines keep 1024-byte alignment");
+};
+
+template <int D>
+struct K2Cfg : TcCfg<D> {
+    using B = TcCfg<D>;
+    static constexpr int NL = D == 32 ? 6 : 3;             // Q landing slots
+    static constexpr int NT = B::NA > B::NO + 1 ? B::NA : B::NO + 1;  // tile-done barriers
+    static constexpr int N2 = OutB<D>::N;
+    static constexpr int BATOM = OutB<D>::BATOM;
+    static constexpr int IMG = OutB<D>::IMG;
+    static constexpr int PRE = (D * D + D) * 4;            // one fp32 prefix state (S, z)
+    // Q ring, operand ring, O staging (4 warps x 32 rows), 2 B images, prefix state
+    static constexpr int PIPE = (NL * B::TB + B::NO * 2 * B::TB + B::TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
+    static constexpr int OFF_CTRL = B::NP * PIPE;
+    static constexpr int FIXED = OFF_CTRL + B::CTRL + 1024;
+    static constexpr int NBAR = 2 * NL + B::NO + NT + B::NA + 4 + 2 * B::NINFO + 1;
+    static constexpr int NINF = 6 * NL + 6 * B::NO + 4 * B::NINFO;
+    static_assert(NBAR <= B::BARS_PER_PIPE && NINF <= B::INFO_PER_PIPE, "control block");
+};
+
+// Named barrier of all transform warps of a CTA (the RoPE table fill, before
+// any work starts; every other hand-over is an mbarrier with a bounded wait).
+constexpr uint32_t kBarTab = 4;
+
+// One pipeline's view of shared memory.
+struct PipeSmem {
+    uint8_t *base;        // the pipeline's rings
+    uint64_t *bars;       // its mbarriers
+    int *info;            // its records
+    volatile int *flags;  // the CTA's: [0] abort
+    uint8_t *ones;        // pass 1: constant B block (all 1.0)
+};
+
+// ---------------------------------------------------------------------------- pass-1 pipeline
 template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(P1<D>::THREADS, 1)
-    partial_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-                      KGeom g, int *watchdog) {
-    using C = P1<D>;
-    constexpr int NP = C::NP, NK = C::NK, NV = C::NV, NO = C::NO, NA = C::NACC, TB = C::TB, ROWB = C::ROWB,
-                  E = D * D + D;
-    constexpr uint32_t IDESC = ptx::idesc_bf16_f32(C::M, C::N, 1, 1);
+struct Pass1 {
+    using C = K1Cfg<D>;
+    static constexpr int NK = C::NK, NV = C::NV, NO = C::NO, NA = C::NA, TB = C::TB, ROWB = C::ROWB, E = C::E;
+    const KGeom &g;
+    PipeSmem ps;
+    int *wd;
+    uint8_t *kring, *vring, *opnd;
+    int *linfo, *oinfo, *cinfo;
+    uint32_t tmem;
 
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = align1024(smem_raw);
-    uint8_t *opnd0 = smem;                         // [NP][NO][K~ | phi]
-    uint8_t *kring0 = opnd0 + NP * NO * 2 * TB;    // [NP][NK][K]
-    uint8_t *vring0 = kring0 + NP * NK * TB;       // [NP][NV][V]
-    uint8_t *ones = vring0 + NP * NV * TB;         // constant B block (above every V tile: positive LBO)
-    uint8_t *ctrl = ones + TB;
-    volatile int *flags = reinterpret_cast<volatile int *>(ctrl + C::BARS);  // [0] abort
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + C::BARS + 4);
-    int *info0 = reinterpret_cast<int *>(ctrl + C::BARS + 16);          // [NP][NK + NO][4]
-    float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // this thread's pipeline
-    const int pipe = warp < 4 * NP ? warp >> 2 : (warp - 4 * NP) % NP;
-    uint8_t *kring = kring0 + pipe * NK * TB;
-    uint8_t *vring = vring0 + pipe * NV * TB;
-    uint8_t *opnd = opnd0 + pipe * NO * 2 * TB;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl) + pipe * C::NBAR;
-    int *linfo = info0 + pipe * 4 * (NK + NO);  // [NK][4] unit, tile, valid, last
-    int *oinfo = linfo + 4 * NK;                 // [NO][4]
-    auto lk = [&](int s) { return kring + s * TB; };
-    auto lv = [&](int s) { return vring + s * TB; };
-    auto ok_ = [&](int s) { return opnd + s * 2 * TB; };
-    auto op_ = [&](int s) { return opnd + s * 2 * TB + TB; };
-    // kfull[s]: K and V of the tile in K slot s have landed (TMA bytes);
-    // kempty[s]: its K has been read (4 transform warps);
-    // tdone[s]: the MMAs of the tile in V slot s are done (1 commit): V slot s
-    //   and that tile's operand slot are free;
-    // ofull[s]: operand slot s is written (4 transform warps)
-    auto kfull = [&](int s) { return ptx::smem_u32(bars + s); };
-    auto kempty = [&](int s) { return ptx::smem_u32(bars + NK + s); };
-    auto tdone = [&](int s) { return ptx::smem_u32(bars + 2 * NK + s); };
-    auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NK + NV + s); };
-    auto accf = [&](int a) { return ptx::smem_u32(bars + 2 * NK + NV + NO + a); };
-    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NK + NV + NO + NA + a); };
-    // drain: one final commit, so that the MMA thread leaves only after all its MMAs are done
-    const uint32_t drain = ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + pipe);
-
-    const int units = g.cpb * g.nblk * g.BH;
-    const int per_c = g.nblk * g.BH;
-    // chunk-index-major order: the short last chunks of every block come last
-    auto decode = [&](int u, int &bh, int &b, int &c) {
-        c = u / per_c;
-        const int rem = u - c * per_c;
-        bh = rem / g.nblk;
-        b = rem - bh * g.nblk;
-    };
-
-    if (tid == 0) {
-        for (int p = 0; p < NP; ++p) {
-            uint64_t *pb = reinterpret_cast<uint64_t *>(ctrl) + p * C::NBAR;
-            for (int s = 0; s < NK; ++s) {
-                ptx::mbar_init(ptx::smem_u32(pb + s), 1);            // kfull: producer (+ TMA bytes)
-                ptx::mbar_init(ptx::smem_u32(pb + NK + s), 4);       // kempty: one arrival per transform warp
-            }
-            for (int s = 0; s < NV; ++s) ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + s), 1);       // tdone: commit
-            for (int s = 0; s < NO; ++s) ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + s), 4);  // ofull
-            for (int a = 0; a < NA; ++a) {
-                ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + NO + a), 1);       // accf: commit
-                ptx::mbar_init(ptx::smem_u32(pb + 2 * NK + NV + NO + NA + a), 4);  // acce: transform warps
-            }
-            ptx::mbar_init(ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + p), 1);  // drain
-        }
-        flags[0] = 0;
-        ptx::fence_mbar_init();
+    __device__ Pass1(const KGeom &g_, const PipeSmem &ps_, int *wd_, uint32_t tmem_base) : g(g_), ps(ps_), wd(wd_) {
+        kring = ps.base;
+        vring = kring + NK * TB;
+        opnd = vring + NV * TB;
+        linfo = ps.info;
+        oinfo = linfo + 5 * NK;
+        cinfo = oinfo + 4 * NO;
+        tmem = tmem_base;
     }
-    if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TCOLS);
-        ptx::tmem_relinquish();
+    __device__ uint8_t *lk(int s) const { return kring + s * TB; }
+    __device__ uint8_t *lv(int s) const { return vring + s * TB; }
+    __device__ uint8_t *ok_(int s) const { return opnd + s * 2 * TB; }
+    __device__ uint8_t *op_(int s) const { return opnd + s * 2 * TB + TB; }
+    // kfull[s]: K and V of the tile in K slot s have landed; kempty[s]: its K is read (4 warps);
+    // tdone[s]: the tile in V slot s is multiplied (V slot and its operand slot free);
+    // ofull[s]: operand slot s written (4 warps); accf/acce: chunk accumulator ready / read;
+    // cfull/cempty: chunk record ring (producer -> epilogue)
+    __device__ uint32_t bar(int i) const { return ptx::smem_u32(ps.bars + i); }
+    __device__ uint32_t kfull(int s) const { return bar(s); }
+    __device__ uint32_t kempty(int s) const { return bar(NK + s); }
+    __device__ uint32_t tdone(int s) const { return bar(2 * NK + s); }
+    __device__ uint32_t ofull(int s) const { return bar(2 * NK + NV + s); }
+    __device__ uint32_t accf(int a) const { return bar(2 * NK + NV + NO + a); }
+    __device__ uint32_t acce(int a) const { return bar(2 * NK + NV + NO + NA + a); }
+    __device__ uint32_t cfull(int i) const { return bar(2 * NK + NV + NO + 2 * NA + i); }
+    __device__ uint32_t cempty(int i) const { return bar(2 * NK + NV + NO + 2 * NA + C::NINFO + i); }
+    __device__ uint32_t drain() const { return bar(2 * NK + NV + NO + 2 * NA + 2 * C::NINFO); }
+
+    __device__ static void init_barriers(uint64_t *b) {
+        auto at = [&](int i) { return ptx::smem_u32(b + i); };
+        for (int s = 0; s < NK; ++s) {
+            ptx::mbar_init(at(s), 1);       // kfull: producer (+ TMA bytes)
+            ptx::mbar_init(at(NK + s), 4);  // kempty: transform warps
+        }
+        for (int s = 0; s < NV; ++s) ptx::mbar_init(at(2 * NK + s), 1);       // tdone: commit
+        for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NK + NV + s), 4);  // ofull
+        for (int a = 0; a < NA; ++a) {
+            ptx::mbar_init(at(2 * NK + NV + NO + a), 1);       // accf: commit
+            ptx::mbar_init(at(2 * NK + NV + NO + NA + a), 4);  // acce: epilogue warps
+        }
+        for (int i = 0; i < C::NINFO; ++i) {
+            ptx::mbar_init(at(2 * NK + NV + NO + 2 * NA + i), 1);            // cfull: producer
+            ptx::mbar_init(at(2 * NK + NV + NO + 2 * NA + C::NINFO + i), 4);  // cempty: epilogue
+        }
+        ptx::mbar_init(at(2 * NK + NV + NO + 2 * NA + 2 * C::NINFO), 1);  // drain
     }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    ptx::tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot + pipe * NA * C::ACOLS;  // this pipeline's accumulators
-    if (tid == 0) griddep_launch_dependents();
 
-    if (warp >= 4 * NP && warp < 5 * NP) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            ptx::tma_prefetch_map(&mk);
-            ptx::tma_prefetch_map(&mv);
-            const uint64_t stream_policy = ptx::l2_evict_first();  // K and V are read once
-            int k = 0;
-            bool ok = true;
-            // the first NP * grid chunks are dealt out statically (chunk blockIdx.x + pipe * grid); after
-            // that each pipeline takes the next unclaimed chunk from a counter, in chunk-index-major
-            // order, so the long chunks go first and every pipeline ends within about one chunk of the
-            // others.  The claim for the following chunk is issued a chunk ahead (its latency hidden).
-            const int first_dyn = NP * gridDim.x;
-            int next = first_dyn + static_cast<int>(atomicAdd(g.sched, 1u));
-            for (int u = blockIdx.x + pipe * gridDim.x; ok && u < units;) {
-                const int u_next = next;
-                if (u_next < units) next = first_dyn + static_cast<int>(atomicAdd(g.sched, 1u));
-                int bh, b, c;
-                decode(u, bh, b, c);
-                const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
-                const int bntok = (fe - fb) * g.HW, cs = c * kChunk;
-                if (cs < bntok) {
-                    const int clen = min(kChunk, bntok - cs), ntiles = (clen + kTile - 1) / kTile;
-                    const int row0 = bh * g.N + fb * g.HW + cs;
-                    for (int t = 0; t < ntiles; ++t, ++k) {
-                        const int sk = k % NK, sv = k % NV;
-                        if ((k >= NK && !ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, watchdog,
-                                                                WD_PARTIAL_EMPTY, kWaitLimitNs)) ||
-                            (k >= NV && !ptx::mbar_wait_bounded(tdone(sv), ((k / NV) - 1) & 1, watchdog,
-                                                                WD_PARTIAL_EMPTY, kWaitLimitNs))) {
-                            ok = false;
-                            break;
-                        }
-                        int *inf = linfo + 4 * sk;
-                        inf[0] = u;
-                        inf[1] = t;
-                        inf[2] = min(kTile, clen - t * kTile);
-                        inf[3] = t == ntiles - 1;
-                        ptx::mbar_arrive_expect_tx(kfull(sk), 2 * TB);
-                        ptx::tma_load_2d_hint(ptx::smem_u32(lk(sk)), &mk, kfull(sk), 0, row0 + t * kTile, stream_policy);
-                        ptx::tma_load_2d_hint(ptx::smem_u32(lv(sv)), &mv, kfull(sk), 0, row0 + t * kTile, stream_policy);
-                    }
-                }
-                u = u_next;
-            }
-            // end marker for the transform warps
-            const int sk = k % NK;
-            if (ok && (k < NK || ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, watchdog, WD_PARTIAL_EMPTY,
-                                                        kWaitLimitNs))) {
-                linfo[4 * sk] = kEndFirst;
-                ptx::mbar_arrive(kfull(sk));
-            }
-        }
-    } else if (warp >= 5 * NP) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int nu = 0;
-            for (int k = 0;; ++k) {
-                const int so = k % NO;
-                if (flags[0] ||
-                    !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_PARTIAL_READY, kWaitLimitNs)) {
-                    flags[0] = 1;
-                    break;
-                }
-                const int *inf = oinfo + 4 * so;
-                const int u = ld_volatile(inf), t = ld_volatile(inf + 1), last = ld_volatile(inf + 3);
-                if (u < 0) break;
-                const int a = nu % NA;
-                if (t == 0 && nu >= NA &&
-                    !ptx::mbar_wait_bounded(acce(a), ((nu / NA) - 1) & 1, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) {
-                    flags[0] = 1;
-                    break;
-                }
-                ptx::tc_fence_after_sync();
-                const int sv = k % NV;  // the tile's V slot (same tile order as the producer)
-                const uint32_t va = ptx::smem_u32(lv(sv));
-                // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones.
-                // Consecutive K steps are 16 token rows (16 * ROWB bytes: ROWB in the address field).
-                const uint64_t ad = ptx::smem_desc(ptx::smem_u32(ok_(so)), TB, 8 * ROWB, C::LAYOUT);
-                const uint64_t bd = ptx::smem_desc(va, ptx::smem_u32(ones) - va, 8 * ROWB, C::LAYOUT);
-                const uint32_t dacc = tmem + a * C::ACOLS;
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    ptx::mma_bf16_ss(dacc, ad + static_cast<uint64_t>(kk * ROWB), bd + static_cast<uint64_t>(kk * ROWB),
-                                     IDESC, (t > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(tdone(sv));
-                if (last) {
-                    ptx::mma_commit(accf(a));
-                    ++nu;
-                }
-            }
-            // every MMA (and the arrivals of the commits above) completes before the CTA's
-            // final barrier and TMEM release, also when a wait gave up
-            ptx::mma_commit(drain);
-            if (!ptx::mbar_wait_bounded(drain, 0, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) flags[0] = 1;
-        }
-    } else {
-        // ------------------------------------------------------------ transform warps: one row per thread
-        const int r = tid & 127, sub = warp & 3;
-        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 128 * NP);
-        {
-            uint4 *o4 = reinterpret_cast<uint4 *>(ones);  // all 1.0, so its swizzle is irrelevant
-            for (int i = tid; i < TB / 16; i += 128 * NP) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-        }
-        ptx::fence_proxy_async_smem();  // the ones block is read by the MMA (async proxy)
-        ptx::named_bar_sync(1, 128 * NP);
+    __device__ int nc_of(int b) const { return units_of_block(g, b, g.nc_first, g.nc_mid, g.nc_last); }
+    __device__ void decode(int u, int &bh, int &b, int &c) const {
+        bh = u / g.U1;
+        unit_block(g, u - bh * g.U1, g.nc_first, g.nc_mid, g.nc_last, b, c);
+    }
 
-        // Chunk epilogue (each warp its TMEM subpartition): accumulator -> chunk
-        // partial.  M = 64 (d = 32): accumulator row m in TMEM lane
-        // (m % 16) + 32 * (m / 16); M = 128 (d = 64): row m in lane m.  Rows
-        // [0, D) hold P, rows [D, 2D) hold phi^T against the ones block, i.e. zp,
-        // in column D.
-        auto epilogue = [&](int u, int a, int ph) {
-            if (!ptx::mbar_wait_bounded(accf(a), ph, watchdog, WD_PARTIAL_ACC, kWaitLimitNs)) flags[0] = 1;
-            ptx::tc_fence_after_sync();
-            constexpr int RPS = D == 32 ? 16 : 32;  // accumulator rows per TMEM subpartition
+    // ------------------------------------------------------------ TMA producer (lanes 0 and 1)
+    // Lane 0 claims chunks, keeps the rings and issues the K loads; lane 1 issues the V
+    // loads of the same tiles.  One thread can keep only so many tile loads moving, so
+    // two issuing threads move twice the bytes.
+    __device__ void producer(const CUtensorMap *mk, const CUtensorMap *mv, int lane) {
+        const bool lead = lane == 0;
+        if (lead) ptx::tma_prefetch_map(mk);
+        else ptx::tma_prefetch_map(mv);
+        const uint64_t policy = ptx::l2_evict_first();  // K and V are read once
+        const int total = g.BH * g.U1;
+        int k = 0, j = 0;
+        bool ok = true;
+        // claims one ahead, so the atomic's latency is hidden
+        int next = lead ? static_cast<int>(atomicAdd(&g.ctl[0], 1u)) : 0;
+        next = __shfl_sync(3u, next, 0);
+        while (ok && next < total) {
+            const int u = next;
+            const int nx = lead ? static_cast<int>(atomicAdd(&g.ctl[0], 1u)) : 0;
+            next = __shfl_sync(3u, nx, 0);
             int bh, b, c;
             decode(u, bh, b, c);
-            float *out = g.part + ((size_t)(bh * g.nblk + b) * g.cpb + c) * E;
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
-            if (sub < 2) {
-                const int m = RPS * sub + lane;  // P row
-#pragma unroll
-                for (int half = 0; half < D / 32; ++half) {
-                    float v[32];
-                    ptx::tmem_ld_32cols(taddr + 32 * half, v);
-                    if (lane < RPS) {
-                        float4 *dst = reinterpret_cast<float4 *>(out + m * D + 32 * half);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
+            const int L = (fe - fb) * g.HW, nt = (L + kTile - 1) / kTile, nc = nc_of(b);
+            const int t_lo = c * nt / nc, t_hi = (c + 1) * nt / nc;
+            const int bb = bh / g.H, hh = bh - bb * g.H;
+            // the chunk's record for the epilogue
+            if (lead) {
+                const int ci = j % C::NINFO;
+                if (j >= C::NINFO &&
+                    !ptx::mbar_wait_bounded(cempty(ci), ((j / C::NINFO) - 1) & 1, wd, WD_P1_INFO, kWaitLimitNs)) {
+                    ok = false;
+                } else {
+                    cinfo[ci] = u;
+                    ptx::mbar_arrive(cfull(ci));
+                }
+            }
+            ok = __shfl_sync(3u, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            ++j;
+            for (int t = t_lo; t < t_hi; ++t, ++k) {
+                const int sk = k % NK, sv = k % NV;
+                const int n = fb * g.HW + t * kTile;  // token (within the head) of the tile's first row
+                if (lead) {
+                    if ((k >= NK && !ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs)) ||
+                        (k >= NV && !ptx::mbar_wait_bounded(tdone(sv), ((k / NV) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs))) {
+                        ok = false;
+                    } else {
+                        int *inf = linfo + 5 * sk;
+                        inf[0] = u;
+                        inf[1] = t - t_lo;
+                        inf[2] = min(kTile, L - t * kTile);
+                        inf[3] = t == t_hi - 1;
+                        inf[4] = n;
+                        ptx::mbar_arrive_expect_tx(kfull(sk), 2 * TB);
                     }
                 }
-            } else {
-                float zv, unused;
-                tmem_ld_2cols(taddr + D, zv, unused);
-                if (lane < RPS) out[D * D + RPS * (sub - 2) + lane] = zv;
+                // both slots are free (and the bytes expected) before either load goes out
+                ok = __shfl_sync(3u, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                const MapCoord mc = map_coord(n, hh, g.swap_q);
+                if (lead) ptx::tma_load_4d_hint(ptx::smem_u32(lk(sk)), mk, kfull(sk), 0, mc.y, mc.z, bb, policy);
+                else ptx::tma_load_4d_hint(ptx::smem_u32(lv(sv)), mv, kfull(sk), 0, mc.y, mc.z, bb, policy);
             }
-            ptx::tc_fence_before_sync();
-            warp_arrive(acce(a), lane);  // accumulator a is free again
-        };
+        }
+        if (!lead) return;
+        // end markers: transform warps (through the landing ring) and epilogue (chunk ring)
+        const int sk = k % NK;
+        bool marked = false;
+        if (ok && (k < NK || ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs))) {
+            linfo[5 * sk] = kEndFirst;
+            ptx::mbar_arrive(kfull(sk));
+            marked = true;
+        }
+        const int ci = j % C::NINFO;
+        if (ok && (j < C::NINFO ||
+                   ptx::mbar_wait_bounded(cempty(ci), ((j / C::NINFO) - 1) & 1, wd, WD_P1_INFO, kWaitLimitNs))) {
+            cinfo[ci] = kEndFirst;
+            ptx::mbar_arrive(cfull(ci));
+        }
+        // No TMA write may still be in flight into this CTA's shared memory when it exits.
+        // Tiles before k - NK were seen landed before their slots were refilled; tile k - NK
+        // too when the end marker went into its slot (that waited for the slot's release).
+        // The end marker moved that slot's phase on, so it must not be waited for again.
+        // (kfull counts the V bytes too.)
+        const int oldest = marked ? k - NK + 1 : k - NK;
+        for (int kk = k - 1; kk >= 0 && kk >= oldest; --kk)
+            ptx::mbar_wait_bounded(kfull(kk % NK), (kk / NK) & 1, wd, WD_P1_FULL, kWaitLimitNs);
+    }
 
-        const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
-        TokPos tp{0, 0, 0};
-        int nu = 0;                               // chunks pushed to the MMA so far
-        int pend_u = -1, pend_a = 0, pend_ph = 0;  // finished chunk whose epilogue is still due
-        int since = 0;                            // tiles pushed since that chunk's last tile
+    // ------------------------------------------------------------ MMA issuer (one thread)
+    __device__ void mma() {
+        constexpr uint32_t IDESC = ptx::idesc_bf16_f32(C::M1, C::N1, 1, 1);
+        int nu = 0;
         for (int k = 0;; ++k) {
-            const int sk = k % NK, so = k % NO;
-            if (flags[0] || !ptx::mbar_wait_bounded(kfull(sk), (k / NK) & 1, watchdog, WD_PARTIAL_FULL, kWaitLimitNs)) {
-                flags[0] = 1;
+            const int so = k % NO;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, wd, WD_P1_READY, kWaitLimitNs)) {
+                ps.flags[0] = 1;
                 break;
             }
-            const int *inf = linfo + 4 * sk;
+            const int *inf = oinfo + 4 * so;
+            const int u = ld_volatile(inf), t = ld_volatile(inf + 1), last = ld_volatile(inf + 3);
+            if (u < 0) break;
+            const int a = nu % NA;
+            if (t == 0 && nu >= NA &&
+                !ptx::mbar_wait_bounded(acce(a), ((nu / NA) - 1) & 1, wd, WD_P1_ACC, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            ptx::tc_fence_after_sync();
+            const int sv = k % NV;  // the tile's V slot (same tile order as the producer)
+            const uint32_t va = ptx::smem_u32(lv(sv));
+            // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones.
+            // Consecutive K steps are 16 token rows (16 * ROWB bytes: ROWB in the address field).
+            const uint64_t ad = ptx::smem_desc(ptx::smem_u32(ok_(so)), TB, 8 * ROWB, C::LAYOUT);
+            const uint64_t bd = ptx::smem_desc(va, ptx::smem_u32(ps.ones) - va, 8 * ROWB, C::LAYOUT);
+            const uint32_t dacc = tmem + a * C::ACOLS;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+                ptx::mma_bf16_ss(dacc, ad + static_cast<uint64_t>(kk * ROWB), bd + static_cast<uint64_t>(kk * ROWB),
+                                 IDESC, (t > 0 || kk > 0) ? 1u : 0u);
+            ptx::mma_commit(tdone(sv));
+            if (last) {
+                ptx::mma_commit(accf(a));
+                ++nu;
+            }
+        }
+        // every MMA (and the arrivals of the commits above) completes before the CTA's
+        // final barrier and TMEM release, also when a wait gave up
+        ptx::mma_commit(drain());
+        if (!ptx::mbar_wait_bounded(drain(), 0, wd, WD_P1_DRAIN, kWaitLimitNs)) ps.flags[0] = 1;
+    }
+
+    // ------------------------------------------------------------ transform warps (one row per thread)
+    __device__ void transform(const RopeTab &tab, int r) {
+        const int lane = r & 31;
+        const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
+        TokPos tp{0, 0, 0};
+        for (int k = 0;; ++k) {
+            const int sk = k % NK, so = k % NO;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(kfull(sk), (k / NK) & 1, wd, WD_P1_FULL, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            const int *inf = linfo + 5 * sk;
             const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
-            const int last = ld_volatile(inf + 3);
+            const int last = ld_volatile(inf + 3), n = ld_volatile(inf + 4);
             // read this row of K; rows past the chunk also clear their V row
             // (the MMA reads V in place: other blocks' tokens must add nothing)
             uint32_t w[D / 2], ph[D / 2];
@@ -537,9 +563,9 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
             ptx::fence_proxy_async_smem();
             if (u >= 0) warp_arrive(kempty(sk), lane);
             // operand slot so was last used by tile k - NO: wait for its MMAs
-            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NV), ((k - NO) / NV) & 1, watchdog,
-                                                   WD_PARTIAL_READY, kWaitLimitNs)) {
-                flags[0] = 1;
+            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NV), ((k - NO) / NV) & 1, wd, WD_P1_READY,
+                                                   kWaitLimitNs)) {
+                ps.flags[0] = 1;
                 break;
             }
             if (u < 0) {  // pass the end on to the MMA issuer, in operand order
@@ -547,13 +573,8 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                 warp_arrive(ofull(so), lane);
                 break;
             }
-            if (t == 0) {
-                int bh, b, c;
-                decode(u, bh, b, c);
-                tp.init(g, block_frame_begin(g, b) * g.HW + c * kChunk + r);
-            } else {
-                tp.advance(g, dx, dy, dt);
-            }
+            if (t == 0) tp.init(g, n + r);
+            else tp.advance(g, dx, dy, dt);
             if (live) {
                 phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
                 store_row<D>(ok_(so), r, w);
@@ -571,309 +592,284 @@ __global__ void __launch_bounds__(P1<D>::THREADS, 1)
                 oi[3] = last;
             }
             warp_arrive(ofull(so), lane);
-            // the previous chunk's epilogue, once its MMAs have had two tiles' time
-            if (pend_u >= 0 && (++since >= 2 || last)) {
-                epilogue(pend_u, pend_a, pend_ph);
-                pend_u = -1;
-            }
-            if (last) {
-                pend_u = u;
-                pend_a = nu % NA;
-                pend_ph = (nu / NA) & 1;
-                since = 0;
-                ++nu;
-            }
         }
-        if (pend_u >= 0 && !flags[0]) epilogue(pend_u, pend_a, pend_ph);
     }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(*tmem_slot, C::TCOLS);
-    }
-}
 
-// ============================================================================ pass 2
-template <int D>
-struct P2 {
-    static constexpr int ROWB = 2 * D;
-    static constexpr int TB = kTile * ROWB;
-    static constexpr int NP = D == 32 ? 2 : 1;          // independent pipelines per CTA (MMA issuers)
-    static constexpr int NL = D == 32 ? 6 : 3;          // Q landing slots per pipeline
-    static constexpr int NO = 2;                        // operand sets per pipeline: q~ | phi(q)
-    static constexpr int NACC = 4;                      // TMEM accumulators per pipeline
-    static constexpr int NT = NACC > NO + 1 ? NACC : NO + 1;  // tile-done barriers per pipeline
-    static constexpr int N = OutB<D>::N;                // num | phi.z_hi | phi.z_lo | pad
-    static constexpr int BATOM = OutB<D>::BATOM;        // one K atom of B (N rows)
-    static constexpr int IMG = OutB<D>::IMG;
-    static constexpr int ACOLS = D == 32 ? 64 : 128;    // TMEM columns per accumulator
-    static constexpr uint32_t TCOLS = NP * NACC * ACOLS;
-    static constexpr uint32_t LAYOUT = D == 32 ? 4u : 2u;
-    static constexpr int PRE = (D * D + D) * 4;         // one fp32 prefix state (S, z)
-    static constexpr int NBAR = 2 * NL + NO + NT + NACC + 6;  // + pfull, pempty, bempty (2 each)
-    static constexpr int CTRL = 2048;
-    static constexpr int BARS = 512;
-    // shared memory of one pipeline, rounded up so every pipeline's swizzled
-    // tiles stay 1024-byte aligned
-    // (+ TB: each epilogue warp's 32-row O staging area for its TMA store)
-    // (the fp32 prefix state is single-buffered: it is turned into the
-    // double-buffered bf16 B operand as soon as it lands)
-    static constexpr int PIPE = (NL * TB + NO * 2 * TB + TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
-    static constexpr int FIXED = NP * PIPE + CTRL + 1024;  // + RoPE table
-    static constexpr int THREADS = 32 * 10 * NP;  // per pipeline: 4 transform, 4 epilogue, producer, MMA warps
-    static_assert(NP * (NBAR + 1) * 8 <= BARS, "mbarriers (+ one drain barrier per pipeline) overflow their area");
-    static_assert(BARS + 16 + NP * 4 * 8 * (NL + NO) <= CTRL, "control block overflow");
-    static_assert(TCOLS <= 512, "TMEM holds 512 columns");
-    static_assert(PIPE % 1024 == 0, "pipelines keep 1024-byte alignment");
+    // ------------------------------------------------------------ epilogue warps: chunk partials
+    // `e` is the thread's index in the 4 epilogue warps; `sub` its warp's TMEM subpartition.
+    __device__ void epilogue(int e, int sub) {
+        const int lane = e & 31;
+        constexpr int RPS = D == 32 ? 16 : 32;  // accumulator rows per TMEM subpartition
+        for (int j = 0;; ++j) {
+            const int ci = j % C::NINFO;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(cfull(ci), (j / C::NINFO) & 1, wd, WD_P1_INFO, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            const int u = ld_volatile(cinfo + ci);
+            warp_arrive(cempty(ci), lane);
+            if (u < 0) break;
+            const int a = j % NA;
+            if (!ptx::mbar_wait_bounded(accf(a), (j / NA) & 1, wd, WD_P1_ACC, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            ptx::tc_fence_after_sync();
+            int bh, b, c;
+            decode(u, bh, b, c);
+            float *out = g.part + (((size_t)bh * g.nblk + b) * g.cpb + c) * E;
+            // M = 64 (d = 32): accumulator row m in TMEM lane (m % 16) + 32 * (m / 16);
+            // M = 128 (d = 64): row m in lane m.  Rows [0, D) hold P, rows [D, 2D) hold
+            // phi^T against the ones block, i.e. zp, in column D.
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
+            if (sub < 2) {
+                const int m = RPS * sub + lane;  // P row
+#pragma unroll
+                for (int half = 0; half < D / 32; ++half) {
+                    float v[32];
+                    ptx::tmem_ld_32cols(taddr + 32 * half, v);
+                    if (lane < RPS) {
+                        float4 *dst = reinterpret_cast<float4 *>(out + m * D + 32 * half);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                }
+            } else {
+                float zv, unused;
+                tmem_ld_2cols(taddr + D, zv, unused);
+                if (lane < RPS) out[D * D + RPS * (sub - 2) + lane] = zv;
+            }
+            ptx::tc_fence_before_sync();
+            warp_arrive(acce(a), lane);  // accumulator a is free again
+        }
+    }
 };
 
-// Persistent, one CTA per SM, NP independent pipelines (see pass 1: two
-// issuing threads keep the tensor core fed).  Pipeline p takes every other
-// group of <= 8 query tiles of one (head, block) from the CTA's static round
-// robin.  Per pipeline: a producer thread bulk-copies each group's fp32
-// prefix state and lands its Q tiles with TMA; four transform warps build the
-// group's bf16 B operand [[S, 0], [0, z_hi z_lo]] from the prefix state, then
-// write [R phi(q) | phi(q)] per tile into an operand ring; an MMA thread
-// computes [Q~ | phi(Q)] x B into one of NACC TMEM accumulators and commits
-// once per tile to a tile-done barrier (which frees the operand slot and tells
-// the epilogue the accumulator is ready); four epilogue warps divide
-// num / (phi(q).z + eps) in fp32, free the accumulator, and each stages its 32
-// bf16 rows in shared memory and stores them with its own TMA store (plain
-// stores for the warp that holds a ragged tile's edge).  `mo` views O with
-// 32-row boxes.
+// ---------------------------------------------------------------------------- pass-2 pipeline
 template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(P2<D>::THREADS, 1)
-    output_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mo, KGeom g,
-                     __nv_bfloat16 *o, int *watchdog) {
-    using C = P2<D>;
-    constexpr int NP = C::NP, NL = C::NL, NO = C::NO, NA = C::NACC, NT = C::NT, TB = C::TB, ROWB = C::ROWB;
-    constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, C::N, 0, 0);
-    const int QG = g.qgt * kTile;  // tokens per group
+struct Pass2 {
+    using C = K2Cfg<D>;
+    static constexpr int NL = C::NL, NO = C::NO, NA = C::NA, NT = C::NT, TB = C::TB, ROWB = C::ROWB, E = C::E;
+    const KGeom &g;
+    PipeSmem ps;
+    int *wd;
+    uint8_t *land, *opnd, *ostg, *bbuf, *pbuf;
+    int *linfo, *oinfo, *tinfo;
+    uint32_t tmem;
 
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = align1024(smem_raw);
-    uint8_t *ctrl = smem + NP * C::PIPE;
-    volatile int *flags = reinterpret_cast<volatile int *>(ctrl + C::BARS);  // [0] abort
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + C::BARS + 4);
-    float2 *s_tab = reinterpret_cast<float2 *>(ctrl + C::CTRL);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // roles: warps [0, 4NP) transform, [4NP, 8NP) epilogue, then NP producers, NP MMA issuers
-    const int pipe = warp < 8 * NP ? (warp >> 2) % NP : (warp - 8 * NP) % NP;
-    uint8_t *pb = smem + pipe * C::PIPE;
-    uint8_t *land = pb;                           // [NL][Q]
-    uint8_t *opnd = land + NL * TB;               // [NO][q~ | phi]
-    uint8_t *ostg = opnd + NO * 2 * TB;           // [4 warps][32 rows] O staging
-    uint8_t *bbuf = ostg + TB;                    // [2][IMG] bf16 B operand
-    uint8_t *pbuf = bbuf + 2 * C::IMG;            // [PRE] fp32 prefix state
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ctrl) + pipe * C::NBAR;
-    int *linfo = reinterpret_cast<int *>(ctrl + C::BARS + 16) + pipe * 8 * (NL + NO);  // [NL][8]
-    int *oinfo = linfo + 8 * NL;                                                     // [NO][8]
-    auto lq = [&](int s) { return land + s * TB; };
-    auto oq = [&](int s) { return opnd + s * 2 * TB; };
-    auto oph = [&](int s) { return opnd + s * 2 * TB + TB; };
-    auto lfull = [&](int s) { return ptx::smem_u32(bars + s); };
-    auto lempty = [&](int s) { return ptx::smem_u32(bars + NL + s); };
-    auto ofull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + s); };
-    auto tdone = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + s); };
-    auto acce = [&](int a) { return ptx::smem_u32(bars + 2 * NL + NO + NT + a); };
-    auto pfull = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + s); };
-    auto pempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + 2 + s); };
-    auto bempty = [&](int s) { return ptx::smem_u32(bars + 2 * NL + NO + NT + NA + 4 + s); };
-    // drain: one final commit, so that the MMA thread leaves only after all its MMAs are done
-    const uint32_t drain = ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + pipe);
-
-    const int units = g.qcpb * g.nblk * g.BH;
-    const int per_q = g.nblk * g.BH;
-    auto decode = [&](int u, int &bh, int &b, int &qc) {
-        qc = u / per_q;
-        const int rem = u - qc * per_q;
-        bh = rem / g.nblk;
-        b = rem - bh * g.nblk;
-    };
-
-    if (tid == 0) {
-        for (int p = 0; p < NP; ++p) {
-            uint64_t *bp = reinterpret_cast<uint64_t *>(ctrl) + p * C::NBAR;
-            for (int s = 0; s < NL; ++s) {
-                ptx::mbar_init(ptx::smem_u32(bp + s), 1);       // lfull: producer + TMA bytes
-                ptx::mbar_init(ptx::smem_u32(bp + NL + s), 4);  // lempty: transform warps
-            }
-            for (int s = 0; s < NO; ++s) ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + s), 4);           // ofull
-            for (int s = 0; s < NT; ++s) ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + s), 1);      // tdone
-            for (int a = 0; a < NA; ++a) ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + a), 4);  // acce
-            for (int s = 0; s < 2; ++s) {
-                ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + s), 1);      // pfull: bulk copy
-                ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + 2 + s), 4);  // pempty: transform warps
-                ptx::mbar_init(ptx::smem_u32(bp + 2 * NL + NO + NT + NA + 4 + s), 1);  // bempty: commit
-            }
-            ptx::mbar_init(ptx::smem_u32(reinterpret_cast<uint64_t *>(ctrl) + NP * C::NBAR + p), 1);  // drain
-        }
-        flags[0] = 0;
-        ptx::fence_mbar_init();
+    __device__ Pass2(const KGeom &g_, const PipeSmem &ps_, int *wd_, uint32_t tmem_base) : g(g_), ps(ps_), wd(wd_) {
+        land = ps.base;
+        opnd = land + NL * TB;
+        ostg = opnd + NO * 2 * TB;
+        bbuf = ostg + TB;
+        pbuf = bbuf + 2 * C::IMG;
+        linfo = ps.info;
+        oinfo = linfo + 6 * NL;
+        tinfo = oinfo + 6 * NO;
+        tmem = tmem_base;
     }
-    if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TCOLS);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before_sync();
-    __syncthreads();
-    ptx::tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot + pipe * NA * C::ACOLS;  // this pipeline's accumulators
+    __device__ uint8_t *lq(int s) const { return land + s * TB; }
+    __device__ uint8_t *oq(int s) const { return opnd + s * 2 * TB; }
+    __device__ uint8_t *oph(int s) const { return opnd + s * 2 * TB + TB; }
+    __device__ uint32_t bar(int i) const { return ptx::smem_u32(ps.bars + i); }
+    __device__ uint32_t lfull(int s) const { return bar(s); }
+    __device__ uint32_t lempty(int s) const { return bar(NL + s); }
+    __device__ uint32_t ofull(int s) const { return bar(2 * NL + s); }
+    __device__ uint32_t tdone(int s) const { return bar(2 * NL + NO + s); }
+    __device__ uint32_t acce(int a) const { return bar(2 * NL + NO + NT + a); }
+    __device__ uint32_t pfull() const { return bar(2 * NL + NO + NT + NA); }
+    __device__ uint32_t pempty() const { return bar(2 * NL + NO + NT + NA + 1); }
+    __device__ uint32_t bempty(int s) const { return bar(2 * NL + NO + NT + NA + 2 + s); }
+    __device__ uint32_t tfull(int i) const { return bar(2 * NL + NO + NT + NA + 4 + i); }
+    __device__ uint32_t tempty(int i) const { return bar(2 * NL + NO + NT + NA + 4 + C::NINFO + i); }
+    __device__ uint32_t drain() const { return bar(2 * NL + NO + NT + NA + 4 + 2 * C::NINFO); }
 
-    // this pipeline's groups: units blockIdx.x + (pipe + NP j) * gridDim.x
-    const int u0 = blockIdx.x + pipe * gridDim.x, ustep = NP * gridDim.x;
-
-    if (warp >= 8 * NP && warp < 9 * NP) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            ptx::tma_prefetch_map(&mq);
-            const uint64_t stream_policy = ptx::l2_evict_first();  // Q is read once
-            int k = 0, nu = 0;
-            bool waited = false, ok = true;
-            auto issue_prefix = [&](int bh, int b, int ord) {
-                // the previous group's prefix has been turned into its B operand
-                if (ord >= 1 &&
-                    !ptx::mbar_wait_bounded(pempty(0), (ord - 1) & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs))
-                    return false;
-                if (!waited) {  // the prefix states are written by the scan
-                    griddep_wait();
-                    waited = true;
-                }
-                ptx::mbar_arrive_expect_tx(pfull(0), C::PRE);
-                ptx::bulk_load(ptx::smem_u32(pbuf), g.prefix + ((size_t)bh * g.nblk + b) * (D * D + D), C::PRE,
-                               pfull(0));
-                return true;
-            };
-            for (int u = u0; ok && u < units; u += ustep) {
-                int bh, b, qc;
-                decode(u, bh, b, qc);
-                const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
-                const int bntok = (fe - fb) * g.HW, qs = qc * QG;
-                if (qs >= bntok) continue;
-                const int qlen = min(QG, bntok - qs), ntiles = (qlen + kTile - 1) / kTile;
-                const int row0 = bh * g.N + fb * g.HW + qs;
-                // the first group's Q tiles go out before waiting on the scan
-                const int early = waited ? 0 : min(ntiles, NL);
-                if (early == 0 && !(ok = issue_prefix(bh, b, nu))) break;
-                for (int t = 0; t < ntiles; ++t, ++k) {
-                    const int sl = k % NL;
-                    if (k >= NL &&
-                        !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY, kWaitLimitNs)) {
-                        ok = false;
-                        break;
-                    }
-                    int *inf = linfo + 8 * sl;
-                    inf[0] = u;
-                    inf[1] = t;
-                    inf[2] = min(kTile, qlen - t * kTile);
-                    inf[3] = nu;
-                    inf[4] = fb * g.HW + qs;  // token index (within the head) of the group's first row
-                    inf[5] = t == ntiles - 1;
-                    ptx::mbar_arrive_expect_tx(lfull(sl), TB);
-                    ptx::tma_load_2d_hint(ptx::smem_u32(lq(sl)), &mq, lfull(sl), 0, row0 + t * kTile, stream_policy);
-                    if (early > 0 && t == early - 1 && !(ok = issue_prefix(bh, b, nu))) break;
-                }
-                ++nu;
-            }
-            // end marker for the transform warps
-            const int sl = k % NL;
-            if (ok && (k < NL || ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, watchdog, WD_OUT_EMPTY,
-                                                        kWaitLimitNs))) {
-                linfo[8 * sl] = kEndFirst;
-                ptx::mbar_arrive(lfull(sl));
-            }
+    __device__ static void init_barriers(uint64_t *b) {
+        auto at = [&](int i) { return ptx::smem_u32(b + i); };
+        for (int s = 0; s < NL; ++s) {
+            ptx::mbar_init(at(s), 1);       // lfull: producer + TMA bytes
+            ptx::mbar_init(at(NL + s), 4);  // lempty: transform warps
         }
-    } else if (warp >= 9 * NP) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            for (int k = 0;; ++k) {
-                const int so = k % NO, a = k % NA;
-                if (flags[0] || !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, watchdog, WD_OUT_READY, kWaitLimitNs)) {
-                    flags[0] = 1;
+        for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NL + s), 4);           // ofull
+        for (int s = 0; s < NT; ++s) ptx::mbar_init(at(2 * NL + NO + s), 1);      // tdone: commit
+        for (int a = 0; a < NA; ++a) ptx::mbar_init(at(2 * NL + NO + NT + a), 4);  // acce: epilogue
+        ptx::mbar_init(at(2 * NL + NO + NT + NA), 1);                              // pfull: bulk copy
+        ptx::mbar_init(at(2 * NL + NO + NT + NA + 1), 4);                          // pempty: transform
+        for (int s = 0; s < 2; ++s) ptx::mbar_init(at(2 * NL + NO + NT + NA + 2 + s), 1);  // bempty: commit
+        for (int i = 0; i < C::NINFO; ++i) {
+            ptx::mbar_init(at(2 * NL + NO + NT + NA + 4 + i), 1);              // tfull: producer
+            ptx::mbar_init(at(2 * NL + NO + NT + NA + 4 + C::NINFO + i), 4);  // tempty: epilogue
+        }
+        ptx::mbar_init(at(2 * NL + NO + NT + NA + 4 + 2 * C::NINFO), 1);  // drain
+    }
+
+    __device__ int ng_of(int b) const { return units_of_block(g, b, g.ng_first, g.ng_mid, g.ng_last); }
+
+    // ------------------------------------------------------------ producer (one thread)
+    __device__ void producer(const CUtensorMap *mq) {
+        ptx::tma_prefetch_map(mq);
+        const uint64_t policy = ptx::l2_evict_first();  // Q is read once
+        const int total = g.BH * g.U2;
+        int k = 0, j = 0, nu = 0, npre = 0;
+        bool ok = true, waited = false;
+        // the group's fp32 prefix state (written by the block scan, the previous kernel)
+        auto issue_prefix = [&](int bh, int b) {
+            if (nu >= 1 && !ptx::mbar_wait_bounded(pempty(), (nu - 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs)) return false;
+            if (!waited) {
+                griddep_wait();
+                waited = true;
+            }
+            ptx::mbar_arrive_expect_tx(pfull(), C::PRE);
+            ptx::bulk_load(ptx::smem_u32(pbuf), g.prefix + ((size_t)bh * g.nblk + b) * E, C::PRE, pfull());
+            ++npre;
+            return true;
+        };
+        int next = static_cast<int>(atomicAdd(&g.ctl[1], 1u));
+        while (ok && next < total) {
+            const int u = next;
+            next = static_cast<int>(atomicAdd(&g.ctl[1], 1u));
+            const int bh = u / g.U2;
+            int b, gi;
+            unit_block(g, u - bh * g.U2, g.ng_first, g.ng_mid, g.ng_last, b, gi);
+            const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
+            const int L = (fe - fb) * g.HW, nt = (L + kTile - 1) / kTile, ng = ng_of(b);
+            const int t_lo = gi * nt / ng, t_hi = (gi + 1) * nt / ng, ntiles = t_hi - t_lo;
+            const int bb = bh / g.H, hh = bh - bb * g.H;
+            // Q tiles do not depend on the prefix: the first few go out before it
+            const int early = min(ntiles, NL);
+            for (int t = 0; t < ntiles; ++t, ++k, ++j) {
+                const int sl = k % NL, ti = j % C::NINFO;
+                if ((k >= NL && !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs)) ||
+                    (j >= C::NINFO &&
+                     !ptx::mbar_wait_bounded(tempty(ti), ((j / C::NINFO) - 1) & 1, wd, WD_P2_INFO, kWaitLimitNs))) {
+                    ok = false;
                     break;
                 }
-                const int *inf = oinfo + 8 * so;
-                const int u = ld_volatile(inf), ord = ld_volatile(inf + 3), last = ld_volatile(inf + 5);
-                if (u < 0) break;
-                if (k >= NA &&
-                    !ptx::mbar_wait_bounded(acce(a), ((k / NA) - 1) & 1, watchdog, WD_OUT_ACCE, kWaitLimitNs)) {
-                    flags[0] = 1;
-                    break;
-                }
-                ptx::tc_fence_after_sync();
-                const uint32_t qa = ptx::smem_u32(oq(so)), pa = ptx::smem_u32(oph(so));
-                const uint32_t ba = ptx::smem_u32(bbuf + (ord & 1) * C::IMG);
-                const uint32_t dacc = tmem + a * C::ACOLS;
+                const int n = fb * g.HW + (t_lo + t) * kTile;
+                const int valid = min(kTile, L - (t_lo + t) * kTile);
+                int *ti_rec = tinfo + 4 * ti;  // for the epilogue
+                ti_rec[0] = n;
+                ti_rec[1] = bh;
+                ti_rec[2] = valid;
+                ptx::mbar_arrive(tfull(ti));
+                int *inf = linfo + 6 * sl;  // for the transform warps
+                inf[0] = u;
+                inf[1] = t;
+                inf[2] = valid;
+                inf[3] = nu;
+                inf[4] = n;
+                inf[5] = t == ntiles - 1;
+                const MapCoord mc = map_coord(n, hh, g.swap_q);
+                ptx::mbar_arrive_expect_tx(lfull(sl), TB);
+                ptx::tma_load_4d_hint(ptx::smem_u32(lq(sl)), mq, lfull(sl), 0, mc.y, mc.z, bb, policy);
+                if (t == early - 1 && !(ok = issue_prefix(bh, b))) break;
+            }
+            ++nu;
+        }
+        // end markers: transform warps (landing ring) and epilogue (tile ring)
+        const int sl = k % NL, ti = j % C::NINFO;
+        bool marked = false;
+        if (ok && (k < NL || ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs))) {
+            linfo[6 * sl] = kEndFirst;
+            ptx::mbar_arrive(lfull(sl));
+            marked = true;
+        }
+        if (ok && (j < C::NINFO ||
+                   ptx::mbar_wait_bounded(tempty(ti), ((j / C::NINFO) - 1) & 1, wd, WD_P2_INFO, kWaitLimitNs))) {
+            tinfo[4 * ti] = kEndFirst;
+            ptx::mbar_arrive(tfull(ti));
+        }
+        // no bulk write may still be in flight into shared memory when the CTA exits (the
+        // same reasoning as in pass 1's producer), including the last prefix copy
+        const int oldest = marked ? k - NL + 1 : k - NL;
+        for (int kk = k - 1; kk >= 0 && kk >= oldest; --kk)
+            ptx::mbar_wait_bounded(lfull(kk % NL), (kk / NL) & 1, wd, WD_P2_FULL, kWaitLimitNs);
+        if (npre > 0) ptx::mbar_wait_bounded(pfull(), (npre - 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs);
+    }
+
+    // ------------------------------------------------------------ MMA issuer (one thread)
+    __device__ void mma() {
+        constexpr uint32_t IDESC = ptx::idesc_bf16_f32(128, C::N2, 0, 0);
+        for (int k = 0;; ++k) {
+            const int so = k % NO, a = k % NA;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(ofull(so), (k / NO) & 1, wd, WD_P2_READY, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            const int *inf = oinfo + 6 * so;
+            const int u = ld_volatile(inf), ord = ld_volatile(inf + 3), last = ld_volatile(inf + 5);
+            if (u < 0) break;
+            if (k >= NA && !ptx::mbar_wait_bounded(acce(a), ((k / NA) - 1) & 1, wd, WD_P2_ACCE, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            ptx::tc_fence_after_sync();
+            const uint32_t qa = ptx::smem_u32(oq(so)), pa = ptx::smem_u32(oph(so));
+            const uint32_t ba = ptx::smem_u32(bbuf + (ord & 1) * C::IMG);
+            const uint32_t dacc = tmem + a * C::ACOLS;
 #pragma unroll
-                for (int kk = 0; kk < 2 * D / 16; ++kk) {
-                    // K atom 0 = q~, K atom 1 = phi(q); +32 B per 16-element K step
-                    const int atom = kk / (D / 16), j = kk % (D / 16);
-                    const uint64_t ad = ptx::smem_desc((atom ? pa : qa) + 32 * j, 16, 8 * ROWB, C::LAYOUT);
-                    const uint64_t bd = ptx::smem_desc(ba + atom * C::BATOM + 32 * j, 16, 8 * ROWB, C::LAYOUT);
-                    ptx::mma_bf16_ss(dacc, ad, bd, IDESC, kk > 0 ? 1u : 0u);
-                }
-                ptx::mma_commit(tdone(k % NT));
-                if (last) ptx::mma_commit(bempty(ord & 1));
+            for (int kk = 0; kk < 2 * D / 16; ++kk) {
+                // K atom 0 = q~, K atom 1 = phi(q); +32 B per 16-element K step
+                const int atom = kk / (D / 16), jj = kk % (D / 16);
+                const uint64_t ad = ptx::smem_desc((atom ? pa : qa) + 32 * jj, 16, 8 * ROWB, C::LAYOUT);
+                const uint64_t bd = ptx::smem_desc(ba + atom * C::BATOM + 32 * jj, 16, 8 * ROWB, C::LAYOUT);
+                ptx::mma_bf16_ss(dacc, ad, bd, IDESC, kk > 0 ? 1u : 0u);
             }
-            // every MMA (and the arrivals of the commits above) completes before the CTA's
-            // final barrier and TMEM release, also when a wait gave up
-            ptx::mma_commit(drain);
-            if (!ptx::mbar_wait_bounded(drain, 0, watchdog, WD_OUT_MMA, kWaitLimitNs)) flags[0] = 1;
+            ptx::mma_commit(tdone(k % NT));
+            if (last) ptx::mma_commit(bempty(ord & 1));
         }
-    } else if (warp < 4 * NP) {
-        // ------------------------------------------------------------ transform warps: one row per thread
-        const int r = tid & 127;
-        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, s_tab, tid, 128 * NP);
-        ptx::named_bar_sync(1, 128 * NP);
+        ptx::mma_commit(drain());
+        if (!ptx::mbar_wait_bounded(drain(), 0, wd, WD_P2_DRAIN, kWaitLimitNs)) ps.flags[0] = 1;
+    }
+
+    // ------------------------------------------------------------ transform warps (one row per thread)
+    __device__ void transform(const RopeTab &tab, int r) {
+        const int lane = r & 31;
         const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
         TokPos tp{0, 0, 0};
         for (int k = 0;; ++k) {
             const int sl = k % NL, so = k % NO;
-            if (flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, watchdog, WD_OUT_FULL, kWaitLimitNs)) {
-                flags[0] = 1;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, wd, WD_P2_FULL, kWaitLimitNs)) {
+                ps.flags[0] = 1;
                 break;
             }
-            const int *inf = linfo + 8 * sl;
-            const int u = ld_volatile(inf);
-            const int t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2), ord = ld_volatile(inf + 3);
-            const int tok0 = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
+            const int *inf = linfo + 6 * sl;
+            const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
+            const int ord = ld_volatile(inf + 3), n = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
             if (u >= 0 && t == 0) {
-                // a new group: build its B operand from the prefix state (the
-                // slot's previous group must be done with it)
+                // a new group: build its B operand from the prefix state (the slot's
+                // previous group must be done with it)
                 const int bs = ord & 1;
-                if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, watchdog, WD_OUT_BREADY,
+                if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, wd, WD_P2_BREADY,
                                                          kWaitLimitNs)) ||
-                    !ptx::mbar_wait_bounded(pfull(0), ord & 1, watchdog, WD_OUT_BREADY, kWaitLimitNs)) {
-                    flags[0] = 1;
+                    !ptx::mbar_wait_bounded(pfull(), ord & 1, wd, WD_P2_BREADY, kWaitLimitNs)) {
+                    ps.flags[0] = 1;
                     break;
                 }
                 const float *pre = reinterpret_cast<const float *>(pbuf);
                 uint4 *dst = reinterpret_cast<uint4 *>(bbuf + bs * C::IMG);
                 for (int item = r; item < C::IMG / 16; item += 128) dst[item] = b_operand_chunk<D>(pre, item);
-                ptx::fence_proxy_async_smem();  // read by the MMA (async proxy); ordered by this tile's ofull
-                warp_arrive(pempty(0), lane);
+                // the next bulk copy into the prefix buffer writes through the async proxy
+                ptx::fence_proxy_async_smem();  // also: the B image is read by the MMA (ordered by ofull)
+                warp_arrive(pempty(), lane);
             }
             uint32_t w[D / 2], ph[D / 2];
             const bool live = u >= 0 && r < valid;
             if (live) load_row<D>(lq(sl), r, w);
-            // the next TMA into this slot writes through the async proxy: order
-            // this thread's generic reads of the slot before it
             ptx::fence_proxy_async_smem();
             if (u >= 0) warp_arrive(lempty(sl), lane);  // landing slot read
             // operand slot so was last used by tile k - NO: wait for its MMAs
-            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NT), ((k - NO) / NT) & 1, watchdog, WD_OUT_READY,
+            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NT), ((k - NO) / NT) & 1, wd, WD_P2_READY,
                                                    kWaitLimitNs)) {
-                flags[0] = 1;
+                ps.flags[0] = 1;
                 break;
             }
             if (u < 0) {  // pass the end on to the MMA issuer, in operand order
-                if (r == 0) oinfo[8 * so] = kEndFirst;
+                if (r == 0) oinfo[6 * so] = kEndFirst;
                 warp_arrive(ofull(so), lane);
                 break;
             }
-            if (t == 0) tp.init(g, tok0 + r);
+            if (t == 0) tp.init(g, n + r);
             else tp.advance(g, dx, dy, dt);
             if (live) {
                 phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
@@ -885,7 +881,7 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
             }
             ptx::fence_proxy_async_smem();
             if (r == 0) {
-                int *oi = oinfo + 8 * so;
+                int *oi = oinfo + 6 * so;
                 oi[0] = u;
                 oi[1] = t;
                 oi[3] = ord;
@@ -893,68 +889,186 @@ __global__ void __launch_bounds__(P2<D>::THREADS, 1)
             }
             warp_arrive(ofull(so), lane);
         }
-    } else {
-        // ------------------------------------------------------------ epilogue warps: one row per thread
-        const int sub = warp & 3, r = 32 * sub + lane;  // tile row = this warp's TMEM subpartition lane
-        uint8_t *stg = ostg + sub * 32 * ROWB;           // this warp's 32 staged rows (swizzled like `mo`)
-        if (lane == 0) ptx::tma_prefetch_map(&mo);
-        const uint64_t stream_policy = ptx::l2_evict_first();  // O is written once
-        int k = 0;
-        for (int u = u0; u < units && !flags[0]; u += ustep) {  // the producer's tile sequence
-            int bh, b, qc;
-            decode(u, bh, b, qc);
-            const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
-            const int bntok = (fe - fb) * g.HW, qs = qc * QG;
-            if (qs >= bntok) continue;
-            const int qlen = min(QG, bntok - qs), ntiles = (qlen + kTile - 1) / kTile;
-            const int row0 = bh * g.N + fb * g.HW + qs;
-            for (int t = 0; t < ntiles; ++t, ++k) {
-                const int a = k % NA;
-                if (!ptx::mbar_wait_bounded(tdone(k % NT), (k / NT) & 1, watchdog, WD_OUT_MMA, kWaitLimitNs)) {
-                    flags[0] = 1;
-                    break;
-                }
-                ptx::tc_fence_after_sync();
-                const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
-                float zh, zl;
-                tmem_ld_2cols(taddr + D, zh, zl);
-                const float inv = __frcp_rn(zh + zl + g.eps);
-                uint32_t ow[D / 2];
-#pragma unroll
-                for (int half = 0; half < D / 32; ++half) {
-                    float v[32];
-                    ptx::tmem_ld_32cols(taddr + 32 * half, v);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) ow[16 * half + q] = pack_bf16x2(v[2 * q] * inv, v[2 * q + 1] * inv);
-                }
-                ptx::tc_fence_before_sync();
-                warp_arrive(acce(a), lane);  // the accumulator is read: the MMA may overwrite it
-                const int valid = min(kTile, qlen - t * kTile);
-                if (32 * sub + 32 <= valid) {
-                    // whole warp in range: stage the 32 rows and store them with TMA
-                    if (lane == 0) ptx::bulk_wait_group_read<0>();  // the previous store has read the staging
-                    __syncwarp();
-                    store_row<D>(stg, lane, ow);
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::tma_store_2d_hint(&mo, ptx::smem_u32(stg), 0, row0 + t * kTile + 32 * sub, stream_policy);
-                        ptx::bulk_commit_group();
-                    }
-                } else if (r < valid) {  // a ragged tile's edge: plain stores of the valid rows
-                    uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)row0 + t * kTile + r) * D);
-#pragma unroll
-                    for (int j = 0; j < D / 8; ++j) dst[j] = make_uint4(ow[4 * j], ow[4 * j + 1], ow[4 * j + 2], ow[4 * j + 3]);
-                }
+    }
+
+    // ------------------------------------------------------------ epilogue warps (one row per thread)
+    // Each warp holds 32 rows of a tile (its TMEM subpartition).  It stages them in shared
+    // memory, then writes them out row-major: one store instruction covers 8 rows (d = 32)
+    // or 4 (d = 64), 512 bytes that are contiguous when rows are.  No TMA store, so no wait
+    // on the copy engine.
+    __device__ void epilogue(__nv_bfloat16 *o, int sub, int lane) {
+        constexpr int CPR = D / 8;                  // 16-byte chunks per row
+        uint8_t *stg = ostg + sub * 32 * ROWB;       // this warp's 32 staged rows (swizzled)
+        for (int k = 0;; ++k) {
+            const int ti = k % C::NINFO, a = k % NA;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(tfull(ti), (k / C::NINFO) & 1, wd, WD_P2_INFO, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
             }
+            const int *rec = tinfo + 4 * ti;
+            const int n = ld_volatile(rec), bh = ld_volatile(rec + 1), valid = ld_volatile(rec + 2);
+            warp_arrive(tempty(ti), lane);
+            if (n < 0) break;
+            if (!ptx::mbar_wait_bounded(tdone(k % NT), (k / NT) & 1, wd, WD_P2_MMA, kWaitLimitNs)) {
+                ps.flags[0] = 1;
+                break;
+            }
+            ptx::tc_fence_after_sync();
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
+            float zh, zl;
+            tmem_ld_2cols(taddr + D, zh, zl);
+            const float inv = __frcp_rn(zh + zl + g.eps);
+            uint32_t ow[D / 2];
+#pragma unroll
+            for (int half = 0; half < D / 32; ++half) {
+                float v[32];
+                ptx::tmem_ld_32cols(taddr + 32 * half, v);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) ow[16 * half + q] = pack_bf16x2(v[2 * q] * inv, v[2 * q + 1] * inv);
+            }
+            ptx::tc_fence_before_sync();
+            warp_arrive(acce(a), lane);  // the accumulator is read: the MMA may overwrite it
+            const int bb = bh / g.H, hh = bh - bb * g.H;
+            __nv_bfloat16 *obase = o + (size_t)bb * g.lo.batch + (size_t)hh * g.lo.head;
+            store_row<D>(stg, lane, ow);
+            __syncwarp();
+#pragma unroll
+            for (int i = lane; i < 32 * CPR; i += 32) {
+                const int row = i / CPR, jj = i - row * CPR, nr = 32 * sub + row;
+                if (nr < valid)
+                    __stcs(reinterpret_cast<uint4 *>(obase + (size_t)(n + nr) * g.lo.tok) + jj,
+                           *reinterpret_cast<const uint4 *>(stg + swz_chunk<D>(row, jj)));
+            }
+            __syncwarp();  // the staging is read before the next tile's rows go in
         }
-        if (lane == 0) ptx::bulk_wait_group<0>();  // stores complete before the CTA exits
+    }
+};
+
+// ---------------------------------------------------------------------------- kernels
+// Shared prologue of both kernels: barriers, TMEM, the RoPE table.  Returns
+// this thread's pipeline index `pipe` and its warp index `pw` inside it.
+template <typename Cfg>
+struct Cta {
+    uint8_t *base, *ctrl;
+    volatile int *flags;
+    float2 *s_tab;
+    uint32_t *tmem_slot;
+    __device__ explicit Cta(uint8_t *raw, int off_ctrl) {
+        base = align1024(raw);
+        ctrl = base + off_ctrl;
+        flags = reinterpret_cast<volatile int *>(ctrl + Cfg::OFF_FLAGS);
+        tmem_slot = reinterpret_cast<uint32_t *>(ctrl + Cfg::OFF_FLAGS + 4);
+        s_tab = reinterpret_cast<float2 *>(ctrl + Cfg::CTRL);
+    }
+    __device__ PipeSmem pipe(int p, int pipe_bytes, uint8_t *ones) const {
+        PipeSmem ps;
+        ps.base = base + p * pipe_bytes;
+        ps.bars = reinterpret_cast<uint64_t *>(ctrl) + p * Cfg::BARS_PER_PIPE;
+        ps.info = reinterpret_cast<int *>(ctrl + Cfg::OFF_INFO) + p * Cfg::INFO_PER_PIPE;
+        ps.flags = flags;
+        ps.ones = ones;
+        return ps;
+    }
+};
+
+// Pass 1: chunk partial states.  Persistent, one CTA per SM, NP pipelines.
+template <int D, int PT, int PY, int PX>
+__global__ void __launch_bounds__(K1Cfg<D>::THREADS, 1)
+    partial_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                      const __grid_constant__ KGeom g, int *watchdog) {
+    using C = K1Cfg<D>;
+    using P = Pass1<D, PT, PY, PX>;
+    extern __shared__ uint8_t smem_raw[];
+    Cta<C> cta(smem_raw, C::OFF_CTRL);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pipe = warp / C::PIPE_WARPS, pw = warp % C::PIPE_WARPS;
+    uint8_t *ones = cta.base + C::OFF_ONES;
+    if (tid == 0) {
+        for (int p = 0; p < C::NP; ++p) P::init_barriers(reinterpret_cast<uint64_t *>(cta.ctrl) + p * C::BARS_PER_PIPE);
+        cta.flags[0] = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(cta.tmem_slot), C::TCOLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem_base = *cta.tmem_slot;
+    if (tid == 0) griddep_launch_dependents();
+    const PipeSmem ps = cta.pipe(pipe, C::PIPE, ones);
+    const uint32_t tmem = tmem_base + pipe * C::NA * C::ACOLS;
+    if (pw < 4) {
+        const int r = tid & 127, ntrans = 128 * C::NP, tt = pipe * 128 + r;
+        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, cta.s_tab, tt, ntrans);
+        uint4 *o4 = reinterpret_cast<uint4 *>(ones);  // all 1.0, so its swizzle is irrelevant
+        for (int i = tt; i < C::TB / 16; i += ntrans) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        ptx::fence_proxy_async_smem();  // the ones block is read by the MMA (async proxy)
+        ptx::named_bar_sync(kBarTab, ntrans);
+        P(g, ps, watchdog, tmem).transform(tab, r);
+    } else if (pw < 8) {
+        P(g, ps, watchdog, tmem).epilogue(tid & 127, warp & 3);
+    } else if (pw == 8) {
+        if (lane < 2) P(g, ps, watchdog, tmem).producer(&mk, &mv, lane);
+    } else if (lane == 0) {
+        P(g, ps, watchdog, tmem).mma();
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after_sync();
-        ptx::tmem_dealloc(*tmem_slot, C::TCOLS);
+        ptx::tmem_dealloc(tmem_base, C::TCOLS);
+    }
+}
+
+// Pass 2: outputs.  Persistent, one CTA per SM, NP pipelines; launched with
+// programmatic dependent launch, it reads the prefix states only after
+// griddepcontrol.wait (the block scan before it has finished).
+template <int D, int PT, int PY, int PX>
+__global__ void __launch_bounds__(K2Cfg<D>::THREADS, 1)
+    output_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ KGeom g, __nv_bfloat16 *o,
+                     int *watchdog) {
+    using C = K2Cfg<D>;
+    using P = Pass2<D, PT, PY, PX>;
+    extern __shared__ uint8_t smem_raw[];
+    Cta<C> cta(smem_raw, C::OFF_CTRL);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pipe = warp / C::PIPE_WARPS, pw = warp % C::PIPE_WARPS;
+    if (tid == 0) {
+        for (int p = 0; p < C::NP; ++p) P::init_barriers(reinterpret_cast<uint64_t *>(cta.ctrl) + p * C::BARS_PER_PIPE);
+        cta.flags[0] = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(cta.tmem_slot), C::TCOLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem_base = *cta.tmem_slot;
+    const PipeSmem ps = cta.pipe(pipe, C::PIPE, nullptr);
+    const uint32_t tmem = tmem_base + pipe * C::NA * C::ACOLS;
+    if (pw < 4) {
+        const int r = tid & 127, ntrans = 128 * C::NP;
+        const RopeTab tab = load_rope_tab<PT, PY, PX>(g, cta.s_tab, pipe * 128 + r, ntrans);
+        ptx::named_bar_sync(kBarTab, ntrans);
+        P(g, ps, watchdog, tmem).transform(tab, r);
+    } else if (pw < 8) {
+        // pass 1 and the scan, which this kernel may overlap, touch neither Q nor O: only
+        // the prefix read (in the producer) waits for them
+        P(g, ps, watchdog, tmem).epilogue(o, warp & 3, lane);
+    } else if (pw == 8) {
+        if (lane == 0) P(g, ps, watchdog, tmem).producer(&mq);
+    } else if (lane == 0) {
+        P(g, ps, watchdog, tmem).mma();
+    }
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc(tmem_base, C::TCOLS);
     }
 }
 

@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA (cp.async.bulk.tensor),
-// tcgen05 (TMEM allocation, MMA, commit, loads) and fences.  No cluster
-// multicast is used anywhere.
+// tcgen05 (TMEM allocation, MMA, commit, loads), GPU-scope flags and fences.
+// No cluster multicast is used anywhere.
 #pragma once
 
 #include <cuda.h>
@@ -100,6 +100,25 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
         : "memory");
 }
+// 4D tile load global -> shared with an L2 cache policy, completion counted on
+// `bar` in bytes (coordinates innermost first).
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y,
+                                                 int z, int w, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w), "l"(policy)
+        : "memory");
+}
+// 4D tile store shared -> global (bulk async group) with an L2 cache policy.
+__device__ __forceinline__ void tma_store_4d_hint(const CUtensorMap *map, uint32_t src, int x, int y, int z, int w,
+                                                  uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y), "r"(z), "r"(w), "l"(policy)
+        : "memory");
+}
 // Contiguous bulk copy global -> shared (16-byte aligned, size multiple of 16),
 // completion counted on `bar` in bytes.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
@@ -133,6 +152,23 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_group() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ------------------------------------------------------------------ global flags
+// Acquire / release accesses at GPU scope, for flags and counters that CTAs
+// of one grid hand to each other.
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Order this thread's generic-proxy global accesses with its later async-proxy
+// ones (bulk copies), and the other way round.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

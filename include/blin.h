@@ -87,6 +87,18 @@ typedef struct {
     float eps;
 } blin_geom;
 
+/* Memory layout of one [B][H][N][d] operand: element (b, h, n, j) sits at
+ * base + b*batch + h*head + n*token + j, strides in elements (d is innermost,
+ * stride 1).  Each stride must be >= d and a multiple of 16 bytes (for bf16: a
+ * multiple of 8 elements); a stride of a dimension of extent 1 is ignored.
+ * Example, a fused QKV projection output [B][N][3][H][d]:
+ *   q = base, k = base + H*d, v = base + 2*H*d,
+ *   {token = 3*H*d, head = d, batch = N*3*H*d}.
+ * Contiguous [B][H][N][d] is {d, N*d, H*N*d}. */
+typedef struct {
+    long long token, head, batch;
+} blin_layout;
+
 typedef struct blin_state blin_state; /* opaque (S, z) cache on one device */
 
 /* ---------------------------------------------------------------- state */
@@ -152,6 +164,20 @@ BLIN_API blin_status blin_prefill(const void *q, const void *k, const void *v, v
                          int B, int H, int d, const blin_geom *g, blin_state *st,
                          void *workspace, size_t ws_bytes, blin_stream stream);
 
+/* blin_prefill on operands in any strided layout (see blin_layout), so a
+ * QKV projection's [B][N][H*d] output (news article, SVDQuant paragraph: the
+ * QKV projections feed this attention) is read in place, with no transpose
+ * into [B][H][N][d]: the tensor-core path addresses it through 4D tensor maps.
+ * qkv_layout applies to q, k and v alike, o_layout to o; NULL means
+ * contiguous [B][H][N][d].  Results are those of blin_prefill on the same
+ * values, bit for bit.  Errors as for blin_prefill, plus BLIN_ERR_SHAPE /
+ * BLIN_ERR_ALIGN for strides that break the rules of blin_layout.  o's rows
+ * must not overlap each other or the inputs. */
+BLIN_API blin_status blin_prefill_strided(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
+                                          int B, int H, int d, const blin_geom *g, const blin_layout *qkv_layout,
+                                          const blin_layout *o_layout, blin_state *st, void *workspace,
+                                          size_t ws_bytes, blin_stream stream);
+
 /* ---------------------------------------------------------------- decode */
 
 /* One autoregressive block, or the part of one that is ready (talk
@@ -174,6 +200,12 @@ BLIN_API blin_status blin_prefill(const void *q, const void *k, const void *v, v
 BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                             int B, int H, int d, const blin_geom *g, blin_state *st, int commit,
                             blin_stream stream);
+
+/* blin_block_step on strided operands (see blin_prefill_strided). */
+BLIN_API blin_status blin_block_step_strided(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
+                                             int B, int H, int d, const blin_geom *g, const blin_layout *qkv_layout,
+                                             const blin_layout *o_layout, blin_state *st, int commit,
+                                             blin_stream stream);
 
 /* ---------------------------------------------------------------- no allocation */
 
@@ -227,15 +259,17 @@ BLIN_API blin_status blin_device_status(int *code);
 
 /* Per-launch timing (profiling aid).  When `events` is non-NULL, the calling
  * thread's next blin_prefill / blin_block_step calls record events[2*i] just
- * before and events[2*i+1] just after launch i on the call's stream, for
- * i = 0 RoPE table, 1 partial states, 2 block scan, 3 output (n >= 8
- * cudaEvent_t handles, owned by the caller).  NULL turns recording off. */
+ * before and events[2*i+1] just after launch slot i on the call's stream
+ * (n >= 8 cudaEvent_t handles, owned by the caller): 0 RoPE table (CUDA-core
+ * path only), 1 partial states, 2 block scan, 3 output.  NULL turns recording
+ * off. */
 BLIN_API blin_status blin_set_timing_events(void *const *events, int n);
 
 /* Number of kernels this library has launched in this process so far (all
  * threads and devices; a profiling aid: the difference across a region counts
  * its launches).  A tensor-core prefill or block step launches 3 (partial
- * states, block scan, output), the general path 4 (RoPE table first). */
+ * states, block scan, output; plus a 16-byte memset of its work counters),
+ * the CUDA-core path 4 (RoPE table first). */
 BLIN_API unsigned long long blin_launch_count(void);
 
 /* Library version string. */

@@ -53,17 +53,35 @@ def ws(B, H, d, g):
     return blin.lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g))
 
 
+def tc_chunks(L, d):
+    """State chunks per block on the tensor-core path: about 5 (d = 32) or 8 (d = 64) tiles of
+    128 tokens each, a function of the block's length and d only."""
+    nt = -(-L // 128)
+    ct = 5 if d == 32 else 8
+    return max(1, -(-nt // ct))
+
+
 def test_workspace_size_formula():
-    # work counters (256 B) + RoPE table + chunk partials + prefix states, each
-    # padded to 256 B, plus 256 B of alignment slack
+    # 256 B of alignment slack, then, each padded to 256 B: the work counters,
+    # the RoPE table, the chunk partials (chunks per block: the larger of the two
+    # paths' counts) and the prefix states
     B, H, d = 1, 70, 32
     g = geom()
     E = d * d + d
     nblk = 21 // 3 + 1
-    cpb = -(-(3 * 30 * 52) // 1024)
+    L = 3 * 30 * 52
+    cpb = max(tc_chunks(L, d), -(-L // 1024))
+    assert cpb == 8
     pad = lambda x: (x + 255) // 256 * 256
-    want = 512 + pad(8 * (21 * 4 + 30 * 6 + 52 * 6 + 1)) + pad(4 * B * H * nblk * cpb * E) + pad(4 * B * H * nblk * E)
+    want = (256 + 256 + pad(8 * (21 * 4 + 30 * 6 + 52 * 6 + 1))
+            + pad(4 * B * H * nblk * cpb * E) + pad(4 * B * H * nblk * E))
     assert ws(B, H, d, g) == want
+
+
+@pytest.mark.parametrize("L,d,want", [(4680, 32, 8), (10800, 32, 17), (1560, 64, 2), (48, 32, 1), (640, 32, 1),
+                                      (641, 32, 2), (1024, 64, 1), (1025, 64, 2)])
+def test_chunk_rule_examples(L, d, want):
+    assert tc_chunks(L, d) == want
 
 
 def test_workspace_size_rejects_bad_shapes():
@@ -139,3 +157,26 @@ def test_state_accessors_reject_null():
 
 def test_version_string():
     assert b"sm_100a" in blin.lib.blin_version()
+
+
+def strided_raw(lq=None, lo=None, dt=1, d=32, H=2, B=1):
+    g = geom(T=4, Hg=4, Wg=4)
+    mk = lambda t: None if t is None else ctypes.byref(blin.Layout(*t))
+    return blin.lib.blin_prefill_strided(FAKE, FAKE, FAKE, FAKE, dt, B, H, d, ctypes.byref(g), mk(lq), mk(lo), None,
+                                         FAKE, 1 << 30, None)
+
+
+@pytest.mark.parametrize("lq,lo,B,code", [
+    ((96, 32, 64 * 96), None, 1, OK),                 # token-interleaved heads, valid
+    ((16, 32 * 64, 2 * 32 * 64), None, 1, SHAPE),     # token stride below d
+    ((36, 32, 64 * 36), None, 1, ALIGN),              # 72-byte rows: not a multiple of 16 bytes
+    (None, (32, 64 * 32, 0), 2, SHAPE),               # batch stride 0 with B = 2
+    (None, (32, 64 * 32, 0), 1, OK),                  # batch stride ignored for B = 1
+])
+def test_strided_layout_checks(lq, lo, B, code):
+    rc = strided_raw(lq=lq, lo=lo, B=B)
+    if code == OK:
+        # valid layouts pass every host check and only then reach the (absent) device
+        assert rc not in (SHAPE, ALIGN, INVALID), blin.lib.blin_last_error().decode()
+    else:
+        assert rc == code, blin.lib.blin_last_error().decode()

@@ -370,3 +370,15 @@ def test_block_step_after_prefill_ending_mid_block(blin):
     S, z = st.to_host()
     assert rel_err(S.numpy().reshape(S_ref.shape), S_ref) <= 5e-3
     assert rel_err(z.numpy().reshape(z_ref.shape), z_ref) <= 1e-5
+
+
+def test_head_subsets_give_the_same_bits(blin):
+    """Heads are independent: a call over all heads equals calls over head subsets, bit for bit
+    (the state chunks of a block depend on the block alone, not on how many heads share a call)."""
+    w = workloads.CONFIGS["480p"].with_(H=24, seed=23)
+    q, k, v = (dev(x, "bf16") for x in workloads.call_tensors(w))
+    want = blin.prefill(q, k, v, (w.T, w.Hg, w.Wg), w.F, w.split, w.theta, w.eps)
+    parts = [blin.prefill(q[:, a:b].contiguous(), k[:, a:b].contiguous(), v[:, a:b].contiguous(),
+                          (w.T, w.Hg, w.Wg), w.F, w.split, w.theta, w.eps) for a, b in ((0, 1), (1, 9), (9, 24))]
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts, dim=1), want)
