@@ -15,6 +15,8 @@ Functions and the passages they follow (SANA-Video pages):
                   encoding paragraph)
   recurrence      state form S_i = S_{i-1} + block contribution, all rows
                   (talk transcript, state review)
+  tconv           causal block temporal convolution with its one-frame cache
+                  (talk transcript, causal-FFN passage)
 
 The RoPE pairing/frequency schedule is a reading of silent pages; it is pinned
 to a library RoPE in the tests, not to the pages.
@@ -63,6 +65,8 @@ def _load():
                                                ctypes.c_double, ctypes.c_double, P, P, P, P, P,
                                                ctypes.c_int]
         lib.blin_oracle_recurrence.restype = ctypes.c_int
+        lib.blin_oracle_tconv.argtypes = [P, P, P, P, L, L, L, L, L, L, P]
+        lib.blin_oracle_tconv.restype = None
         _lib = lib
     return _lib
 
@@ -171,3 +175,20 @@ def recurrence(q, k, v, pos, blk, split, theta: float, eps: float, S_in=None, z_
     if rc != 0:
         raise MemoryError("oracle recurrence: allocation failed")
     return out, S_out, z_out
+
+
+def tconv(x, w, bias, F: int, t0: int = 0, prev=None):
+    """Causal block temporal convolution over frames t0 .. t0+T-1.
+
+    x: [B, T, HW, C] values (float32); w: [C, 3] taps (previous, current, next);
+    bias: [C] or None; prev: [B, HW, C] previous frame (the cache) or None.
+    Returns (y [B, T, HW, C] float64, the call's last frame [B, HW, C] float64)."""
+    x = _f32(x)
+    B, T, HW, C = x.shape
+    w = np.ascontiguousarray(w, dtype=np.float64).reshape(C, 3)
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64).reshape(C)
+    prev = None if prev is None else np.ascontiguousarray(prev, dtype=np.float64).reshape(B, HW, C)
+    y = np.zeros((B, T, HW, C), np.float64)
+    _load().blin_oracle_tconv(_p(x), _p(prev), _p(w), _p(bias), B, T, HW, C, int(t0), int(F), _p(y))
+    last = x[:, -1].astype(np.float64) if T > 0 else prev
+    return y, last

@@ -222,3 +222,37 @@ int blin_oracle_recurrence(const float *q, const float *k, const float *v, const
     }
     return rc ? -1 : 0;
 }
+
+/* Causal block temporal convolution of the Mix-FFN, with its one-frame cache.
+ * (Talk transcript, causal-FFN passage: in causal training a zero token is put
+ * between two blocks, so that block i cannot see block i+1; block i+1 must
+ * see block i, so block i's last token is cached and put in front of block
+ * i+1.)  Per batch entry, spatial position s and channel c, with taps
+ * w[c] = (previous, current, next):
+ *   y[t] = w[c][0] * x[t-1] + w[c][1] * x[t] + w[c][2] * x[t+1] + bias[c]
+ * where x[t-1] is the previous frame (from this call, or `prev` -- the cache,
+ * the last frame of the previous call -- for the call's first frame; zero
+ * before the video's first frame), and x[t+1] is the next frame only when it
+ * lies in the same block of F frames (t_abs / F) and in this call; otherwise
+ * zero (the pad between blocks).
+ *   x: [B][T][HW][C] float32 values of absolute frames t0 .. t0+T-1
+ *   prev: [B][HW][C] (frame t0-1) or NULL for zero
+ *   w: [C][3], bias: [C] or NULL;  y: [B][T][HW][C] */
+void blin_oracle_tconv(const float *x, const double *prev, const double *w, const double *bias, long B,
+                       long T, long HW, long C, long t0, long F, double *y) {
+    for (long b = 0; b < B; ++b)
+        for (long t = 0; t < T; ++t)
+            for (long s = 0; s < HW; ++s)
+                for (long c = 0; c < C; ++c) {
+                    const long ta = t0 + t;
+                    double xp = 0.0, xn = 0.0;
+                    if (t > 0)
+                        xp = (double)x[((b * T + t - 1) * HW + s) * C + c];
+                    else if (ta > 0 && prev != NULL)
+                        xp = prev[(b * HW + s) * C + c];
+                    if (t + 1 < T && (ta + 1) / F == ta / F) xn = (double)x[((b * T + t + 1) * HW + s) * C + c];
+                    const double xc = (double)x[((b * T + t) * HW + s) * C + c];
+                    y[((b * T + t) * HW + s) * C + c] =
+                        w[3 * c] * xp + w[3 * c + 1] * xc + w[3 * c + 2] * xn + (bias ? bias[c] : 0.0);
+                }
+}

@@ -23,6 +23,7 @@ from typing import Optional, Tuple
 import numpy as np
 
 TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_QSCALE, TENSOR_KSCALE = 0, 1, 2, 3, 4
+TENSOR_CONV_X, TENSOR_CONV_W, TENSOR_CONV_BIAS = 5, 6, 7
 
 
 @dataclass(frozen=True)
@@ -149,3 +150,54 @@ def as_storage(x: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "f32":
         return np.ascontiguousarray(x, dtype=np.float32)
     return f32_to_bf16_bits(x)
+
+
+# ----------------------------------------------------------------------------- temporal convolution
+@dataclass(frozen=True)
+class ConvWorkload:
+    """Causal block temporal convolution of the Mix-FFN: tokens [B, T*Hg*Wg, C] of
+    C channels (channels innermost), blocks of F frames.  C defaults to the
+    attention's width (70 heads x 32); the pages do not state the FFN's own."""
+
+    name: str
+    B: int
+    C: int
+    T: int
+    Hg: int
+    Wg: int
+    F: int
+    dtype: str = "bf16"
+    seed: int = 0
+    t0: int = 0
+
+    @property
+    def HW(self) -> int:
+        return self.Hg * self.Wg
+
+    @property
+    def N(self) -> int:
+        return self.T * self.HW
+
+    def with_(self, **kw) -> "ConvWorkload":
+        return replace(self, **kw)
+
+
+CONV_CONFIGS = {
+    "conv-tiny": ConvWorkload("conv-tiny", B=2, C=16, T=7, Hg=3, Wg=5, F=3, dtype="f32"),
+    "conv-480p": ConvWorkload("conv-480p", B=1, C=2240, T=21, Hg=30, Wg=52, F=3),
+}
+
+
+def conv_tensors(w: ConvWorkload):
+    """x [B, T, HW, C] (one stream per frame, keyed by the absolute frame), taps [C, 3]
+    and bias [C] (float32 values; x bf16-representable for bf16 workloads)."""
+    frames = []
+    for t in range(w.t0, w.t0 + w.T):
+        x = _normal(w.seed, TENSOR_CONV_X, t, (w.B, 1, w.HW, w.C))
+        if w.dtype == "bf16":
+            x = bf16_bits_to_f32(f32_to_bf16_bits(x))
+        frames.append(x)
+    x = np.ascontiguousarray(np.concatenate(frames, axis=1)) if frames else np.zeros((w.B, 0, w.HW, w.C), np.float32)
+    taps = 0.5 * _normal(w.seed, TENSOR_CONV_W, 0, (w.C, 3))
+    bias = 0.1 * _normal(w.seed, TENSOR_CONV_BIAS, 0, (w.C,))
+    return x, taps, bias
