@@ -17,7 +17,9 @@ oracle's CPU rate and the SM clocks seen while timing, plus sub-records:
                commit=1): per-block latency percentiles, the same calls
                replayed as one CUDA graph, device memory after every block;
   denoise      16 blocks, each denoised by 4 read-only block steps (fresh
-               Q/K/V, commit=0) and then committed once, replayed as a graph.
+               Q/K/V, commit=0) and then committed once, replayed as a graph;
+  tconv        the Mix-FFN's causal block temporal convolution over the same
+               latent video (C = 2240 channels), bytes against the HBM peak.
 
 With N > 1 GPUs every rank runs its own independent copy of the workload (weak
 scaling; heads and videos never exchange data) and each time is the max over
@@ -596,6 +598,51 @@ def measure_decode(args, w, torch, blin, world, rank, clk, denoise_steps: int = 
     return rec
 
 
+def measure_tconv(args, w, torch, blin, world, rank, clk):
+    """Causal block temporal convolution over a whole latent video (one call): time per call,
+    and algorithmic bytes (x read, y written) against the HBM peak."""
+    wr = w.with_(seed=w.seed + rank)
+    x, taps, bias = workloads.conv_tensors(wr)
+    dt_t = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    xd = torch.from_numpy(x.reshape(w.B, -1, w.C)).to("cuda", dt_t)
+    td, bd = torch.from_numpy(taps).cuda(), torch.from_numpy(bias).cuda()
+    yd = torch.empty_like(xd)
+    geom = blin._geom(w.T, w.Hg, w.Wg, w.F, (0, 0, 0), 1e4, 0.0)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    cargs = (ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(td.data_ptr()), ctypes.c_void_p(bd.data_ptr()),
+             ctypes.c_void_p(yd.data_ptr()), blin.BF16 if w.dtype == "bf16" else blin.F32, w.B, w.C,
+             ctypes.byref(geom), None, 0, stream)
+    call = blin.lib.blin_tconv
+
+    def step():
+        rc = call(*cargs)
+        if rc != 0:
+            raise RuntimeError(blin.lib.blin_last_error().decode())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall = time.time()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clk.timed(t_wall, time.time())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    elem = 2 if w.dtype == "bf16" else 4
+    alg = 2 * w.B * w.N * w.C * elem
+    peak, peak_kind = hbm_peak()
+    return {"workload": f"{w.name}: causal block temporal convolution, B={w.B} C={w.C} {w.dtype}, latent "
+                        f"{w.T}x{w.Hg}x{w.Wg}, blocks of {w.F} frames, taps (previous, current, next) + bias",
+            "ms_per_step": ms, "value": w.B * w.N * w.C / (ms * 1e-3), "unit": "token*channels/s",
+            "roofline": {"bound": "hbm", "kernel": "tconv", "achieved": alg / (ms * 1e-3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": alg / (ms * 1e-3) / 1e9 / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": alg}}
+
+
 def run_blin(args):
     torch, blin, world, rank, local = _load_blin(args)
     main_name = "720p" if args.config == "all" else args.config
@@ -624,6 +671,7 @@ def run_blin(args):
             subs["decode"] = measure_decode(args, workloads.CONFIGS["decode"], torch, blin, world, rank, clk, 0)
             subs["denoise"] = measure_decode(args, workloads.CONFIGS["decode"].with_(steps=16), torch, blin, world,
                                              rank, clk, 4)
+            subs["tconv"] = measure_tconv(args, workloads.CONV_CONFIGS["conv-480p"], torch, blin, world, rank, clk)
         time.sleep(0.25)
     line = {"metric": main.pop("metric"), "value": main.pop("value"), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main.pop("ms_per_step"),

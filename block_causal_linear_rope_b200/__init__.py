@@ -21,7 +21,7 @@ from typing import Optional, Sequence, Tuple
 
 import torch
 
-__all__ = ["BlinError", "BlockState", "Layout", "prefill", "block_step", "workspace_size", "device_status",
+__all__ = ["BlinError", "BlockState", "TConvState", "tconv", "Layout", "prefill", "block_step", "workspace_size", "device_status",
            "last_path", "LaunchTimer", "KERNELS", "lib", "LIB_PATH", "F32", "BF16"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -84,6 +84,16 @@ def _load() -> ctypes.CDLL:
     L.blin_prefill_static.restype = I
     L.blin_prefill_static_capacity.argtypes = []
     L.blin_prefill_static_capacity.restype = S
+    L.blin_tconv_state_init.argtypes = [I, I, I, I, I, P, ctypes.POINTER(P)]
+    L.blin_tconv_state_free.argtypes = [P]
+    L.blin_tconv_state_reset.argtypes = [P, P]
+    L.blin_tconv_state_frame.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(I)]
+    L.blin_tconv_state_bytes.argtypes = [P]
+    L.blin_tconv_state_bytes.restype = S
+    L.blin_tconv.argtypes = [P, P, P, P, I, I, I, ctypes.POINTER(Geom), P, I, P]
+    for fn in ("blin_tconv_state_init", "blin_tconv_state_free", "blin_tconv_state_reset", "blin_tconv_state_frame",
+               "blin_tconv"):
+        getattr(L, fn).restype = I
     L.blin_launch_count.argtypes = []
     L.blin_launch_count.restype = ctypes.c_ulonglong
     for fn in ("blin_state_init", "blin_state_free", "blin_state_reset", "blin_state_tensors",
@@ -350,3 +360,79 @@ def device_status() -> int:
 def launch_count() -> int:
     """Kernels this library has launched in this process so far."""
     return int(lib.blin_launch_count())
+
+
+# ----------------------------------------------------------------------------- temporal convolution
+class TConvState:
+    """One-frame cache of the causal block temporal convolution: [B, Hg*Wg, C]."""
+
+    def __init__(self, B: int, C: int, Hg: int, Wg: int, dtype=torch.bfloat16, stream=None):
+        self.B, self.C, self.Hg, self.Wg = B, C, Hg, Wg
+        self.dtype = dtype
+        h = ctypes.c_void_p()
+        dt = BF16 if dtype == torch.bfloat16 else F32
+        _check(lib.blin_tconv_state_init(B, C, Hg, Wg, dt, _stream(stream), ctypes.byref(h)))
+        self._h = h
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise BlinError(-6, "state already freed")
+        return self._h
+
+    def free(self) -> None:
+        if self._h is not None:
+            _check(lib.blin_tconv_state_free(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            if getattr(self, "_h", None) is not None:
+                lib.blin_tconv_state_free(self._h)
+        except Exception:
+            pass
+
+    @property
+    def t_next(self) -> int:
+        t = ctypes.c_int()
+        _check(lib.blin_tconv_state_frame(self.handle, None, ctypes.byref(t)))
+        return t.value
+
+    @property
+    def nbytes(self) -> int:
+        return int(lib.blin_tconv_state_bytes(self.handle))
+
+    def reset(self, stream=None) -> None:
+        _check(lib.blin_tconv_state_reset(self.handle, _stream(stream)))
+
+    def frame_ptr(self) -> int:
+        """Device address of the cached frame [B, Hg*Wg, C]."""
+        ptr = ctypes.c_void_p()
+        _check(lib.blin_tconv_state_frame(self.handle, ctypes.byref(ptr), None))
+        return int(ptr.value)
+
+
+def tconv(x: torch.Tensor, taps: torch.Tensor, bias: Optional[torch.Tensor], grid: Sequence[int], block_frames: int,
+          state: Optional[TConvState] = None, commit: bool = True, out: Optional[torch.Tensor] = None,
+          stream=None) -> torch.Tensor:
+    """Causal block temporal convolution of x [B, T*Hg*Wg, C] (frame-major tokens, channels
+    innermost) with taps [C, 3] (previous, current, next) and bias [C] (fp32, or None).
+    With a state, the call continues its video and (if commit) updates its cache; without
+    one it is the start of a video and nothing is cached."""
+    if x.dim() != 3 or not x.is_contiguous() or not x.is_cuda:
+        raise ValueError("x must be a contiguous CUDA [B, T*Hg*Wg, C] tensor")
+    B, N, C = x.shape
+    T, Hg, Wg = (int(v) for v in grid)
+    if N != T * Hg * Wg:
+        raise ValueError(f"N={N} but T*Hg*Wg={T * Hg * Wg}")
+    taps = taps.to(device=x.device, dtype=torch.float32).contiguous()
+    if bias is not None:
+        bias = bias.to(device=x.device, dtype=torch.float32).contiguous()
+    if out is None:
+        out = torch.empty_like(x)
+    g = _geom(T, Hg, Wg, block_frames, (0, 0, 0), 1e4, 0.0)
+    _check(lib.blin_tconv(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(taps.data_ptr()),
+                          None if bias is None else ctypes.c_void_p(bias.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                          _dtype_code(x), B, C, ctypes.byref(g), None if state is None else state.handle,
+                          1 if (commit and state is not None) else 0, _stream(stream)))
+    return out

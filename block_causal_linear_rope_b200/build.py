@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libblin.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["blin_api.cu", "blin_kernels.cu", "blin_noalloc.cu"]
+SOURCES = ["blin_api.cu", "blin_kernels.cu", "blin_noalloc.cu", "blin_tconv.cu"]
 FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",

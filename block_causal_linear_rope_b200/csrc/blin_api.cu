@@ -266,6 +266,8 @@ static thread_local cudaEvent_t const *g_timing = nullptr;
 // Kernels this library has launched in this process (all threads, all devices).
 static std::atomic<unsigned long long> g_launches{0};
 
+void blin::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 static void mark(int i, bool after, cudaStream_t s) {
     if (g_timing != nullptr) cudaEventRecord(g_timing[2 * i + (after ? 1 : 0)], s);
 }
@@ -288,7 +290,8 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
         CUtensorMap mq, mk, mv;
         int sk = 0, sv = 0;
         const int B = g.BH / g.H;
-        if (!make_map4(&mq, q, g.lq, B, g.H, g.N, d, kTile, &g.swap_q) ||
+        // pass 2 lands Q in spans of tiles (one box each: 256 rows at d = 32, 128 at d = 64)
+        if (!make_map4(&mq, q, g.lq, B, g.H, g.N, d, d == 32 ? 2 * kTile : kTile, &g.swap_q) ||
             !make_map4(&mk, k, g.lq, B, g.H, g.N, d, kTile, &sk) || !make_map4(&mv, v, g.lq, B, g.H, g.N, d, kTile, &sv))
             return fail(BLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or strides rejected)");
         // both kernels hand out their work through counters that start at zero

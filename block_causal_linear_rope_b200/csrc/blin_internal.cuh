@@ -152,4 +152,7 @@ struct ContextCache {
 // Records `msg` as this thread's blin_last_error() text and returns `st`.
 blin_status set_last_error(blin_status st, const char *msg);
 
+// Counts one kernel launch in blin_launch_count().
+void note_launch();
+
 }  // namespace blin

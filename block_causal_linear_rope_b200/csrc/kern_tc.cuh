@@ -313,7 +313,11 @@ struct K1Cfg : TcCfg<D> {
 template <int D>
 struct K2Cfg : TcCfg<D> {
     using B = TcCfg<D>;
-    static constexpr int NL = D == 32 ? 6 : 3;             // Q landing slots
+    // Q lands in slots of SPAN consecutive tiles, one TMA box each: the copy engine moves
+    // a 16-KB box in about the time of an 8-KB one, so fewer, larger boxes move more bytes
+    static constexpr int SPAN = D == 32 ? 2 : 1;           // tiles per Q landing slot
+    static constexpr int NLS = 3;                          // Q landing slots
+    static constexpr int NL = NLS * SPAN;                  // Q tiles in the landing ring
     static constexpr int NT = B::NA > B::NO + 1 ? B::NA : B::NO + 1;  // tile-done barriers
     static constexpr int N2 = OutB<D>::N;
     static constexpr int BATOM = OutB<D>::BATOM;
@@ -323,8 +327,8 @@ struct K2Cfg : TcCfg<D> {
     static constexpr int PIPE = (NL * B::TB + B::NO * 2 * B::TB + B::TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
     static constexpr int OFF_CTRL = B::NP * PIPE;
     static constexpr int FIXED = OFF_CTRL + B::CTRL + 1024;
-    static constexpr int NBAR = 2 * NL + B::NO + NT + B::NA + 4 + 2 * B::NINFO + 1;
-    static constexpr int NINF = 6 * NL + 6 * B::NO + 4 * B::NINFO;
+    static constexpr int NBAR = 2 * NLS + B::NO + NT + B::NA + 4 + 2 * B::NINFO + 1;
+    static constexpr int NINF = 8 * NLS + 6 * B::NO + 4 * B::NINFO;
     static_assert(NBAR <= B::BARS_PER_PIPE && NINF <= B::INFO_PER_PIPE, "control block");
 };
 
@@ -649,7 +653,8 @@ struct Pass1 {
 template <int D, int PT, int PY, int PX>
 struct Pass2 {
     using C = K2Cfg<D>;
-    static constexpr int NL = C::NL, NO = C::NO, NA = C::NA, NT = C::NT, TB = C::TB, ROWB = C::ROWB, E = C::E;
+    static constexpr int NL = C::NL, NLS = C::NLS, SPAN = C::SPAN, NO = C::NO, NA = C::NA, NT = C::NT, TB = C::TB,
+                         ROWB = C::ROWB, E = C::E;
     const KGeom &g;
     PipeSmem ps;
     int *wd;
@@ -664,53 +669,55 @@ struct Pass2 {
         bbuf = ostg + TB;
         pbuf = bbuf + 2 * C::IMG;
         linfo = ps.info;
-        oinfo = linfo + 6 * NL;
+        oinfo = linfo + 8 * NLS;
         tinfo = oinfo + 6 * NO;
         tmem = tmem_base;
     }
-    __device__ uint8_t *lq(int s) const { return land + s * TB; }
+    __device__ uint8_t *lq(int s) const { return land + s * SPAN * TB; }
     __device__ uint8_t *oq(int s) const { return opnd + s * 2 * TB; }
     __device__ uint8_t *oph(int s) const { return opnd + s * 2 * TB + TB; }
     __device__ uint32_t bar(int i) const { return ptx::smem_u32(ps.bars + i); }
     __device__ uint32_t lfull(int s) const { return bar(s); }
-    __device__ uint32_t lempty(int s) const { return bar(NL + s); }
-    __device__ uint32_t ofull(int s) const { return bar(2 * NL + s); }
-    __device__ uint32_t tdone(int s) const { return bar(2 * NL + NO + s); }
-    __device__ uint32_t acce(int a) const { return bar(2 * NL + NO + NT + a); }
-    __device__ uint32_t pfull() const { return bar(2 * NL + NO + NT + NA); }
-    __device__ uint32_t pempty() const { return bar(2 * NL + NO + NT + NA + 1); }
-    __device__ uint32_t bempty(int s) const { return bar(2 * NL + NO + NT + NA + 2 + s); }
-    __device__ uint32_t tfull(int i) const { return bar(2 * NL + NO + NT + NA + 4 + i); }
-    __device__ uint32_t tempty(int i) const { return bar(2 * NL + NO + NT + NA + 4 + C::NINFO + i); }
-    __device__ uint32_t drain() const { return bar(2 * NL + NO + NT + NA + 4 + 2 * C::NINFO); }
+    __device__ uint32_t lempty(int s) const { return bar(NLS + s); }
+    __device__ uint32_t ofull(int s) const { return bar(2 * NLS + s); }
+    __device__ uint32_t tdone(int s) const { return bar(2 * NLS + NO + s); }
+    __device__ uint32_t acce(int a) const { return bar(2 * NLS + NO + NT + a); }
+    __device__ uint32_t pfull() const { return bar(2 * NLS + NO + NT + NA); }
+    __device__ uint32_t pempty() const { return bar(2 * NLS + NO + NT + NA + 1); }
+    __device__ uint32_t bempty(int s) const { return bar(2 * NLS + NO + NT + NA + 2 + s); }
+    __device__ uint32_t tfull(int i) const { return bar(2 * NLS + NO + NT + NA + 4 + i); }
+    __device__ uint32_t tempty(int i) const { return bar(2 * NLS + NO + NT + NA + 4 + C::NINFO + i); }
+    __device__ uint32_t drain() const { return bar(2 * NLS + NO + NT + NA + 4 + 2 * C::NINFO); }
 
     __device__ static void init_barriers(uint64_t *b) {
         auto at = [&](int i) { return ptx::smem_u32(b + i); };
-        for (int s = 0; s < NL; ++s) {
-            ptx::mbar_init(at(s), 1);       // lfull: producer + TMA bytes
-            ptx::mbar_init(at(NL + s), 4);  // lempty: transform warps
+        for (int s = 0; s < NLS; ++s) {
+            ptx::mbar_init(at(s), 1);        // lfull: producer + TMA bytes
+            ptx::mbar_init(at(NLS + s), 4);  // lempty: transform warps
         }
-        for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NL + s), 4);           // ofull
-        for (int s = 0; s < NT; ++s) ptx::mbar_init(at(2 * NL + NO + s), 1);      // tdone: commit
-        for (int a = 0; a < NA; ++a) ptx::mbar_init(at(2 * NL + NO + NT + a), 4);  // acce: epilogue
-        ptx::mbar_init(at(2 * NL + NO + NT + NA), 1);                              // pfull: bulk copy
-        ptx::mbar_init(at(2 * NL + NO + NT + NA + 1), 4);                          // pempty: transform
-        for (int s = 0; s < 2; ++s) ptx::mbar_init(at(2 * NL + NO + NT + NA + 2 + s), 1);  // bempty: commit
+        for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NLS + s), 4);           // ofull
+        for (int s = 0; s < NT; ++s) ptx::mbar_init(at(2 * NLS + NO + s), 1);      // tdone: commit
+        for (int a = 0; a < NA; ++a) ptx::mbar_init(at(2 * NLS + NO + NT + a), 4);  // acce: epilogue
+        ptx::mbar_init(at(2 * NLS + NO + NT + NA), 1);                              // pfull: bulk copy
+        ptx::mbar_init(at(2 * NLS + NO + NT + NA + 1), 4);                          // pempty: transform
+        for (int s = 0; s < 2; ++s) ptx::mbar_init(at(2 * NLS + NO + NT + NA + 2 + s), 1);  // bempty: commit
         for (int i = 0; i < C::NINFO; ++i) {
-            ptx::mbar_init(at(2 * NL + NO + NT + NA + 4 + i), 1);              // tfull: producer
-            ptx::mbar_init(at(2 * NL + NO + NT + NA + 4 + C::NINFO + i), 4);  // tempty: epilogue
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + i), 1);              // tfull: producer
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + C::NINFO + i), 4);  // tempty: epilogue
         }
-        ptx::mbar_init(at(2 * NL + NO + NT + NA + 4 + 2 * C::NINFO), 1);  // drain
+        ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + 2 * C::NINFO), 1);  // drain
     }
 
     __device__ int ng_of(int b) const { return units_of_block(g, b, g.ng_first, g.ng_mid, g.ng_last); }
 
     // ------------------------------------------------------------ producer (one thread)
+    // Q goes out in spans of SPAN tiles of one group, one TMA box (SPAN * 128 rows) per
+    // landing slot; rows past the group's block are masked by the transform warps.
     __device__ void producer(const CUtensorMap *mq) {
         ptx::tma_prefetch_map(mq);
         const uint64_t policy = ptx::l2_evict_first();  // Q is read once
         const int total = g.BH * g.U2;
-        int k = 0, j = 0, nu = 0, npre = 0;
+        int kp = 0, j = 0, nu = 0, npre = 0;
         bool ok = true, waited = false;
         // the group's fp32 prefix state (written by the block scan, the previous kernel)
         auto issue_prefix = [&](int bh, int b) {
@@ -734,43 +741,51 @@ struct Pass2 {
             const int fb = block_frame_begin(g, b), fe = block_frame_end(g, b);
             const int L = (fe - fb) * g.HW, nt = (L + kTile - 1) / kTile, ng = ng_of(b);
             const int t_lo = gi * nt / ng, t_hi = (gi + 1) * nt / ng, ntiles = t_hi - t_lo;
+            const int nspans = (ntiles + SPAN - 1) / SPAN;
             const int bb = bh / g.H, hh = bh - bb * g.H;
-            // Q tiles do not depend on the prefix: the first few go out before it
-            const int early = min(ntiles, NL);
-            for (int t = 0; t < ntiles; ++t, ++k, ++j) {
-                const int sl = k % NL, ti = j % C::NINFO;
-                if ((k >= NL && !ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs)) ||
-                    (j >= C::NINFO &&
-                     !ptx::mbar_wait_bounded(tempty(ti), ((j / C::NINFO) - 1) & 1, wd, WD_P2_INFO, kWaitLimitNs))) {
+            // Q spans do not depend on the prefix: the first few go out before it
+            const int early = min(nspans, NLS);
+            for (int p = 0; p < nspans; ++p, ++kp) {
+                const int sl = kp % NLS;
+                if (kp >= NLS && !ptx::mbar_wait_bounded(lempty(sl), ((kp / NLS) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
-                const int n = fb * g.HW + (t_lo + t) * kTile;
-                const int valid = min(kTile, L - (t_lo + t) * kTile);
-                int *ti_rec = tinfo + 4 * ti;  // for the epilogue
-                ti_rec[0] = n;
-                ti_rec[1] = bh;
-                ti_rec[2] = valid;
-                ptx::mbar_arrive(tfull(ti));
-                int *inf = linfo + 6 * sl;  // for the transform warps
+                const int t0 = p * SPAN, n = fb * g.HW + (t_lo + t0) * kTile;  // span's first tile and token
+                // one record per tile for the epilogue
+                for (int h = 0; h < SPAN && t0 + h < ntiles && ok; ++h, ++j) {
+                    const int ti = j % C::NINFO;
+                    if (j >= C::NINFO &&
+                        !ptx::mbar_wait_bounded(tempty(ti), ((j / C::NINFO) - 1) & 1, wd, WD_P2_INFO, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    int *ti_rec = tinfo + 4 * ti;
+                    ti_rec[0] = n + h * kTile;
+                    ti_rec[1] = bh;
+                    ti_rec[2] = min(kTile, L - (t_lo + t0 + h) * kTile);
+                    ptx::mbar_arrive(tfull(ti));
+                }
+                if (!ok) break;
+                int *inf = linfo + 8 * sl;  // for the transform warps
                 inf[0] = u;
-                inf[1] = t;
-                inf[2] = valid;
+                inf[1] = t0;
+                inf[2] = ntiles;
                 inf[3] = nu;
                 inf[4] = n;
-                inf[5] = t == ntiles - 1;
+                inf[5] = L - (t_lo + t0) * kTile;  // rows of the span inside the block (may exceed the span)
                 const MapCoord mc = map_coord(n, hh, g.swap_q);
-                ptx::mbar_arrive_expect_tx(lfull(sl), TB);
+                ptx::mbar_arrive_expect_tx(lfull(sl), SPAN * TB);
                 ptx::tma_load_4d_hint(ptx::smem_u32(lq(sl)), mq, lfull(sl), 0, mc.y, mc.z, bb, policy);
-                if (t == early - 1 && !(ok = issue_prefix(bh, b))) break;
+                if (p == early - 1 && !(ok = issue_prefix(bh, b))) break;
             }
             ++nu;
         }
         // end markers: transform warps (landing ring) and epilogue (tile ring)
-        const int sl = k % NL, ti = j % C::NINFO;
+        const int sl = kp % NLS, ti = j % C::NINFO;
         bool marked = false;
-        if (ok && (k < NL || ptx::mbar_wait_bounded(lempty(sl), ((k / NL) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs))) {
-            linfo[6 * sl] = kEndFirst;
+        if (ok && (kp < NLS || ptx::mbar_wait_bounded(lempty(sl), ((kp / NLS) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs))) {
+            linfo[8 * sl] = kEndFirst;
             ptx::mbar_arrive(lfull(sl));
             marked = true;
         }
@@ -779,11 +794,12 @@ struct Pass2 {
             tinfo[4 * ti] = kEndFirst;
             ptx::mbar_arrive(tfull(ti));
         }
-        // no bulk write may still be in flight into shared memory when the CTA exits (the
-        // same reasoning as in pass 1's producer), including the last prefix copy
-        const int oldest = marked ? k - NL + 1 : k - NL;
-        for (int kk = k - 1; kk >= 0 && kk >= oldest; --kk)
-            ptx::mbar_wait_bounded(lfull(kk % NL), (kk / NL) & 1, wd, WD_P2_FULL, kWaitLimitNs);
+        // No bulk write may still be in flight into shared memory when the CTA exits: the
+        // last landing of each slot (the end marker's slot was seen released, and its phase
+        // moved on) and the last prefix copy.
+        const int oldest = marked ? kp - NLS + 1 : kp - NLS;
+        for (int kk = kp - 1; kk >= 0 && kk >= oldest; --kk)
+            ptx::mbar_wait_bounded(lfull(kk % NLS), (kk / NLS) & 1, wd, WD_P2_FULL, kWaitLimitNs);
         if (npre > 0) ptx::mbar_wait_bounded(pfull(), (npre - 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs);
     }
 
@@ -827,67 +843,88 @@ struct Pass2 {
         const int lane = r & 31;
         const int dx = kTile % g.Wg, dy = (kTile / g.Wg) % g.Hg, dt = kTile / g.HW;
         TokPos tp{0, 0, 0};
-        for (int k = 0;; ++k) {
-            const int sl = k % NL, so = k % NO;
-            if (ps.flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (k / NL) & 1, wd, WD_P2_FULL, kWaitLimitNs)) {
+        int k = 0;  // tiles handed to the MMA so far
+        for (int kp = 0;; ++kp) {
+            const int sl = kp % NLS;
+            if (ps.flags[0] || !ptx::mbar_wait_bounded(lfull(sl), (kp / NLS) & 1, wd, WD_P2_FULL, kWaitLimitNs)) {
                 ps.flags[0] = 1;
                 break;
             }
-            const int *inf = linfo + 6 * sl;
-            const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
-            const int ord = ld_volatile(inf + 3), n = ld_volatile(inf + 4), last = ld_volatile(inf + 5);
-            if (u >= 0 && t == 0) {
-                // a new group: build its B operand from the prefix state (the slot's
-                // previous group must be done with it)
-                const int bs = ord & 1;
-                if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, wd, WD_P2_BREADY,
-                                                         kWaitLimitNs)) ||
-                    !ptx::mbar_wait_bounded(pfull(), ord & 1, wd, WD_P2_BREADY, kWaitLimitNs)) {
+            const int *inf = linfo + 8 * sl;
+            const int u = ld_volatile(inf), t0 = ld_volatile(inf + 1), ntiles = ld_volatile(inf + 2);
+            const int ord = ld_volatile(inf + 3), n = ld_volatile(inf + 4), rows = ld_volatile(inf + 5);
+            if (u < 0) {  // pass the end on to the MMA issuer, in operand order
+                const int so = k % NO;
+                if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NT), ((k - NO) / NT) & 1, wd, WD_P2_READY,
+                                                       kWaitLimitNs)) {
                     ps.flags[0] = 1;
                     break;
                 }
-                const float *pre = reinterpret_cast<const float *>(pbuf);
-                uint4 *dst = reinterpret_cast<uint4 *>(bbuf + bs * C::IMG);
-                for (int item = r; item < C::IMG / 16; item += 128) dst[item] = b_operand_chunk<D>(pre, item);
-                // the next bulk copy into the prefix buffer writes through the async proxy
-                ptx::fence_proxy_async_smem();  // also: the B image is read by the MMA (ordered by ofull)
-                warp_arrive(pempty(), lane);
-            }
-            uint32_t w[D / 2], ph[D / 2];
-            const bool live = u >= 0 && r < valid;
-            if (live) load_row<D>(lq(sl), r, w);
-            ptx::fence_proxy_async_smem();
-            if (u >= 0) warp_arrive(lempty(sl), lane);  // landing slot read
-            // operand slot so was last used by tile k - NO: wait for its MMAs
-            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NT), ((k - NO) / NT) & 1, wd, WD_P2_READY,
-                                                   kWaitLimitNs)) {
-                ps.flags[0] = 1;
-                break;
-            }
-            if (u < 0) {  // pass the end on to the MMA issuer, in operand order
                 if (r == 0) oinfo[6 * so] = kEndFirst;
                 warp_arrive(ofull(so), lane);
                 break;
             }
-            if (t == 0) tp.init(g, n + r);
-            else tp.advance(g, dx, dy, dt);
-            if (live) {
-                phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
-                store_row<D>(oq(so), r, w);
-                store_row<D>(oph(so), r, ph);
-            } else {  // rows past the group: finite values, outputs not stored
-                zero_row<D>(oq(so), r);
-                zero_row<D>(oph(so), r);
+            const int hmax = min(SPAN, ntiles - t0);
+            bool abort = false;
+            for (int h = 0; h < hmax; ++h, ++k) {
+                const int t = t0 + h, so = k % NO;
+                const int valid = min(kTile, rows - h * kTile);
+                if (t == 0) {
+                    // a new group: build its B operand from the prefix state (the slot's
+                    // previous group must be done with it)
+                    const int bs = ord & 1;
+                    if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, wd, WD_P2_BREADY,
+                                                             kWaitLimitNs)) ||
+                        !ptx::mbar_wait_bounded(pfull(), ord & 1, wd, WD_P2_BREADY, kWaitLimitNs)) {
+                        abort = true;
+                        break;
+                    }
+                    const float *pre = reinterpret_cast<const float *>(pbuf);
+                    uint4 *dst = reinterpret_cast<uint4 *>(bbuf + bs * C::IMG);
+                    for (int item = r; item < C::IMG / 16; item += 128) dst[item] = b_operand_chunk<D>(pre, item);
+                    // the next bulk copy into the prefix buffer writes through the async proxy
+                    ptx::fence_proxy_async_smem();  // also: the B image is read by the MMA (ordered by ofull)
+                    warp_arrive(pempty(), lane);
+                }
+                uint32_t w[D / 2], ph[D / 2];
+                const bool live = r < valid;
+                if (live) load_row<D>(lq(sl) + h * TB, r, w);
+                if (h == hmax - 1) {
+                    // the next TMA into this slot writes through the async proxy: order this
+                    // thread's generic reads of the slot before it
+                    ptx::fence_proxy_async_smem();
+                    warp_arrive(lempty(sl), lane);  // landing slot read
+                }
+                // operand slot so was last used by tile k - NO: wait for its MMAs
+                if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NT), ((k - NO) / NT) & 1, wd, WD_P2_READY,
+                                                       kWaitLimitNs)) {
+                    abort = true;
+                    break;
+                }
+                if (t == 0) tp.init(g, n + h * kTile + r);
+                else tp.advance(g, dx, dy, dt);
+                if (live) {
+                    phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
+                    store_row<D>(oq(so), r, w);
+                    store_row<D>(oph(so), r, ph);
+                } else {  // rows past the group: finite values, outputs not stored
+                    zero_row<D>(oq(so), r);
+                    zero_row<D>(oph(so), r);
+                }
+                ptx::fence_proxy_async_smem();
+                if (r == 0) {
+                    int *oi = oinfo + 6 * so;
+                    oi[0] = u;
+                    oi[1] = t;
+                    oi[3] = ord;
+                    oi[5] = t == ntiles - 1;
+                }
+                warp_arrive(ofull(so), lane);
             }
-            ptx::fence_proxy_async_smem();
-            if (r == 0) {
-                int *oi = oinfo + 6 * so;
-                oi[0] = u;
-                oi[1] = t;
-                oi[3] = ord;
-                oi[5] = last;
+            if (abort) {
+                ps.flags[0] = 1;
+                break;
             }
-            warp_arrive(ofull(so), lane);
         }
     }
 

@@ -207,6 +207,50 @@ BLIN_API blin_status blin_block_step_strided(const void *q, const void *k, const
                                              const blin_layout *o_layout, blin_state *st, int commit,
                                              blin_stream stream);
 
+/* ---------------------------------------------------------------- causal temporal convolution */
+
+/* The Mix-FFN's causal block temporal convolution and its one-frame cache
+ * (talk transcript, causal-FFN passage: in causal training a zero token sits
+ * between two blocks, so no block sees the next one; a block sees the
+ * previous block through that block's last token, which is cached and put in
+ * front of the block).  Per batch entry, pixel and channel c, with taps
+ * w[c] = (previous, current, next):
+ *   y[t] = w[c][0] * x[t-1] + w[c][1] * x[t] + w[c][2] * x[t+1] + bias[c]
+ * x[t-1] is the previous frame: from the call, or for the call's first frame
+ * from the cache (zero before the video's first frame); x[t+1] counts only when
+ * it lies in the same block of F = block_frames frames and in the call, else
+ * zero.  Accumulation in fp32 in the order bias, previous, current, next;
+ * outputs have the input dtype (bf16 rounded to nearest even). */
+typedef struct blin_tconv_state blin_tconv_state; /* the last frame seen, [B][Hgt*Wid][C], and t_next */
+
+/* Allocate a zeroed cache on the current device (t_next = 0).  C must be a
+ * multiple of 8.  Its size is fixed: one frame, whatever the video length. */
+BLIN_API blin_status blin_tconv_state_init(int B, int C, int Hgt, int Wid, blin_dtype dt, blin_stream stream,
+                                           blin_tconv_state **out);
+/* Free the cache (waits for the last call that used it).  NULL is a no-op. */
+BLIN_API blin_status blin_tconv_state_free(blin_tconv_state *st);
+/* Zero the cache and set t_next = 0 (a new video). */
+BLIN_API blin_status blin_tconv_state_reset(blin_tconv_state *st, blin_stream stream);
+/* Device pointer of the cached frame and the next absolute frame index (either may be NULL). */
+BLIN_API blin_status blin_tconv_state_frame(const blin_tconv_state *st, void **frame, int *t_next);
+/* Bytes of the cached frame: B * Hgt * Wid * C * element size. */
+BLIN_API size_t blin_tconv_state_bytes(const blin_tconv_state *st);
+
+/* Temporal convolution of frames [t0, t0 + g->T) of a latent video.
+ *   x, y   device [B][g->T * g->Hgt * g->Wid][C] tokens (frame-major, channels
+ *          innermost) of dtype dt, 16-byte aligned; y must not overlap x
+ *   taps   device fp32 [C][3]; bias device fp32 [C] or NULL
+ *   g      T, Hgt, Wid and block_frames are used (the RoPE fields are not)
+ *   st     NULL: the call is the start of a video (t0 = 0).  Otherwise t0 =
+ *          st's t_next and the call's first frame sees the cached frame.
+ *   commit 1 (needs st): the cache takes the call's last frame, t_next += T;
+ *          0: the cache is only read (a denoising pass of the same block).
+ * Calls split at block boundaries, each committed, give bitwise the outputs of
+ * one call over the same frames.  A call that ends inside a block gives its
+ * last frame no next neighbour (that frame is not given yet). */
+BLIN_API blin_status blin_tconv(const void *x, const float *taps, const float *bias, void *y, blin_dtype dt, int B,
+                                int C, const blin_geom *g, blin_tconv_state *st, int commit, blin_stream stream);
+
 /* ---------------------------------------------------------------- no allocation */
 
 /* blin_prefill for callers that cannot allocate device memory (the method on
