@@ -17,6 +17,8 @@ Functions and the passages they follow (SANA-Video pages):
                   (talk transcript, state review)
   tconv           causal block temporal convolution with its one-frame cache
                   (talk transcript, causal-FFN passage)
+  nvfp4_decode    NVFP4 block-scaled 4-bit values (news article, NVFP4 /
+                  SVDQuant paragraph): E2M1 codes x E4M3 block scale x global
 
 The RoPE pairing/frequency schedule is a reading of silent pages; it is pinned
 to a library RoPE in the tests, not to the pages.
@@ -67,6 +69,12 @@ def _load():
         lib.blin_oracle_recurrence.restype = ctypes.c_int
         lib.blin_oracle_tconv.argtypes = [P, P, P, P, L, L, L, L, L, L, P]
         lib.blin_oracle_tconv.restype = None
+        lib.blin_oracle_e2m1.argtypes = [ctypes.c_int]
+        lib.blin_oracle_e2m1.restype = ctypes.c_double
+        lib.blin_oracle_e4m3.argtypes = [ctypes.c_int]
+        lib.blin_oracle_e4m3.restype = ctypes.c_double
+        lib.blin_oracle_nvfp4_decode.argtypes = [P, P, L, ctypes.c_int, ctypes.c_double, P]
+        lib.blin_oracle_nvfp4_decode.restype = None
         _lib = lib
     return _lib
 
@@ -192,3 +200,31 @@ def tconv(x, w, bias, F: int, t0: int = 0, prev=None):
     _load().blin_oracle_tconv(_p(x), _p(prev), _p(w), _p(bias), B, T, HW, C, int(t0), int(F), _p(y))
     last = x[:, -1].astype(np.float64) if T > 0 else prev
     return y, last
+
+
+def e2m1(code: int) -> float:
+    return float(_load().blin_oracle_e2m1(int(code)))
+
+
+def e4m3(code: int) -> float:
+    return float(_load().blin_oracle_e4m3(int(code)))
+
+
+def nvfp4_decode(data, scale, d: int, global_scale: float) -> np.ndarray:
+    """data [..., d/2] uint8, scale [..., d/16] uint8 -> float64 values [..., d]."""
+    data = np.ascontiguousarray(data, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.uint8)
+    lead = data.shape[:-1]
+    rows = int(np.prod(lead)) if lead else 1
+    out = np.empty(lead + (d,), np.float64)
+    _load().blin_oracle_nvfp4_decode(_p(data), _p(scale), rows, int(d), float(global_scale), _p(out))
+    return out
+
+
+def exact_f32(x64: np.ndarray) -> np.ndarray:
+    """float32 copy of float64 values that float32 holds exactly (raises otherwise), for the
+    float32-input oracle routines."""
+    x32 = np.ascontiguousarray(x64, dtype=np.float32)
+    if not np.array_equal(x32.astype(np.float64), x64):
+        raise ValueError("values are not exact in float32")
+    return x32

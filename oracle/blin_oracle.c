@@ -256,3 +256,34 @@ void blin_oracle_tconv(const float *x, const double *prev, const double *w, cons
                         w[3 * c] * xp + w[3 * c + 1] * xc + w[3 * c + 2] * xn + (bias ? bias[c] : 0.0);
                 }
 }
+
+/* NVFP4 block-scaled 4-bit inputs (news article, NVFP4 / SVDQuant paragraph:
+ * the QKV projections run in NVFP4).  Element i of a d-vector is an E2M1 code
+ * (bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa) in nibble i of
+ * the row's d/2 bytes (even elements in the low nibble); each run of 16
+ * consecutive elements shares one E4M3 scale byte (bit 7 sign, bits 6..3
+ * exponent with bias 7, bits 2..0 mantissa; no infinities, 0x7f/0xff NaN);
+ * the tensor has one global scale.  value = e2m1 * e4m3 * global. */
+double blin_oracle_e2m1(int code) {
+    const int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+double blin_oracle_e4m3(int code) {
+    const int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Dequantise rows x rows of d elements: data [rows][d/2], scale [rows][d/16] -> out [rows][d]. */
+void blin_oracle_nvfp4_decode(const unsigned char *data, const unsigned char *scale, long rows, int d,
+                              double global, double *out) {
+    for (long r = 0; r < rows; ++r)
+        for (int i = 0; i < d; ++i) {
+            const int byte = data[r * (d / 2) + i / 2];
+            const int code = (i & 1) ? (byte >> 4) & 15 : byte & 15;
+            out[r * d + i] = blin_oracle_e2m1(code) * blin_oracle_e4m3(scale[r * (d / 16) + i / 16]) * global;
+        }
+}

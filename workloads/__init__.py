@@ -24,6 +24,8 @@ import numpy as np
 
 TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_QSCALE, TENSOR_KSCALE = 0, 1, 2, 3, 4
 TENSOR_CONV_X, TENSOR_CONV_W, TENSOR_CONV_BIAS = 5, 6, 7
+# The 4-bit E2M1 magnitudes, by code (bit 3 is the sign): a format definition.
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float32)
 
 
 @dataclass(frozen=True)
@@ -201,3 +203,54 @@ def conv_tensors(w: ConvWorkload):
     taps = 0.5 * _normal(w.seed, TENSOR_CONV_W, 0, (w.C, 3))
     bias = 0.1 * _normal(w.seed, TENSOR_CONV_BIAS, 0, (w.C,))
     return x, taps, bias
+
+
+# ----------------------------------------------------------------------------- NVFP4 inputs
+def nvfp4_encode(x: np.ndarray, global_scale: float):
+    """Quantise float32 [..., d] to NVFP4: per 16 consecutive elements an E4M3 scale
+    (the block's max |x| / (6 * global), rounded to E4M3 by torch), then each element
+    x / (scale * global) rounded to the nearest E2M1 value (ties to the even code).
+    Returns (data [..., d/2] uint8, even elements in the low nibble;
+    scale [..., d/16] uint8).  A number-format conversion of the inputs only."""
+    import torch
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    d = x.shape[-1]
+    blocks = x.reshape(x.shape[:-1] + (d // 16, 16))
+    amax = np.abs(blocks).max(axis=-1)
+    s_f = (amax / (6.0 * global_scale)).astype(np.float32)
+    s_t = torch.from_numpy(s_f).to(torch.float8_e4m3fn)
+    scale = s_t.view(torch.uint8).numpy().copy()
+    s_val = s_t.float().numpy().astype(np.float64)
+    denom = s_val[..., None] * float(global_scale)
+    v = np.divide(blocks, denom, out=np.zeros(blocks.shape, np.float64), where=denom > 0)
+    mag = np.minimum(np.abs(v), 6.0)
+    grid = E2M1_GRID.astype(np.float64)
+    dist = np.abs(mag[..., None] - grid)
+    idx = np.argmin(dist, axis=-1)  # the lower code on a tie between neighbours
+    nxt = np.minimum(idx + 1, 7)
+    tie_up = (idx % 2 == 1) & (np.take_along_axis(dist, nxt[..., None], -1)[..., 0] == np.take_along_axis(dist, idx[..., None], -1)[..., 0])
+    idx = np.where(tie_up, nxt, idx)  # ties go to the even code
+    code = (idx | np.where((v < 0) & (idx > 0), 8, 0)).astype(np.uint8).reshape(x.shape)
+    data = (code[..., 0::2] | (code[..., 1::2] << 4)).astype(np.uint8)
+    return data, scale
+
+
+def nvfp4_global_scale(x: np.ndarray) -> float:
+    """A power-of-two global scale putting the largest block scale near E4M3's top (448):
+    powers of two keep every dequantised value exact in float32 and bfloat16."""
+    amax = float(np.abs(x).max())
+    if amax == 0.0:
+        return 1.0
+    return float(2.0 ** np.ceil(np.log2(amax / (6.0 * 448.0))))
+
+
+def nvfp4_call_tensors(w: Workload):
+    """Q, K, V of a call as NVFP4: ((data, scale, global) x 3), drawn like call_tensors in float32
+    and then quantised; one global scale per tensor."""
+    out = []
+    w32 = w.with_(dtype="f32")
+    for x in call_tensors(w32):
+        g = nvfp4_global_scale(x)
+        data, scale = nvfp4_encode(x, g)
+        out.append((data, scale, g))
+    return tuple(out)
