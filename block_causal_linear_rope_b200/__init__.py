@@ -21,7 +21,8 @@ from typing import Optional, Sequence, Tuple
 
 import torch
 
-__all__ = ["BlinError", "BlockState", "TConvState", "tconv", "Layout", "prefill", "block_step", "workspace_size", "device_status",
+__all__ = ["BlinError", "BlockState", "TConvState", "tconv", "Layout", "prefill", "prefill_nvfp4", "block_step_nvfp4",
+           "Nvfp4Tensor", "block_step", "workspace_size", "device_status",
            "last_path", "LaunchTimer", "KERNELS", "lib", "LIB_PATH", "F32", "BF16"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +36,10 @@ _STATUS = {0: "BLIN_OK", -1: "BLIN_ERR_INVALID_ARG", -2: "BLIN_ERR_SHAPE", -3: "
 
 class Layout(ctypes.Structure):
     _fields_ = [("token", ctypes.c_longlong), ("head", ctypes.c_longlong), ("batch", ctypes.c_longlong)]
+
+
+class Nvfp4(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("global_scale", ctypes.c_float)]
 
 
 class BlinError(RuntimeError):
@@ -84,6 +89,11 @@ def _load() -> ctypes.CDLL:
     L.blin_prefill_static.restype = I
     L.blin_prefill_static_capacity.argtypes = []
     L.blin_prefill_static_capacity.restype = S
+    NP_ = ctypes.POINTER(Nvfp4)
+    L.blin_prefill_nvfp4.argtypes = [NP_, NP_, NP_, P, I, I, I, ctypes.POINTER(Geom), P, P, S, P]
+    L.blin_prefill_nvfp4.restype = I
+    L.blin_block_step_nvfp4.argtypes = [NP_, NP_, NP_, P, I, I, I, ctypes.POINTER(Geom), P, I, P]
+    L.blin_block_step_nvfp4.restype = I
     L.blin_tconv_state_init.argtypes = [I, I, I, I, I, P, ctypes.POINTER(P)]
     L.blin_tconv_state_free.argtypes = [P]
     L.blin_tconv_state_reset.argtypes = [P, P]
@@ -435,4 +445,72 @@ def tconv(x: torch.Tensor, taps: torch.Tensor, bias: Optional[torch.Tensor], gri
                           None if bias is None else ctypes.c_void_p(bias.data_ptr()), ctypes.c_void_p(out.data_ptr()),
                           _dtype_code(x), B, C, ctypes.byref(g), None if state is None else state.handle,
                           1 if (commit and state is not None) else 0, _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------------------- NVFP4 inputs
+class Nvfp4Tensor:
+    """An NVFP4 [B, H, N, d] operand on the device: packed E2M1 codes [B, H, N, d/2] (uint8,
+    even element in the low nibble), E4M3 block scales [B, H, N, d/16] (uint8, one per 16
+    elements; stored in an allocation padded to 16 bytes) and a global scale."""
+
+    def __init__(self, data: torch.Tensor, scale: torch.Tensor, global_scale: float):
+        if data.dtype != torch.uint8 or scale.dtype != torch.uint8 or data.dim() != 4 or scale.dim() != 4:
+            raise ValueError("data and scale must be 4D uint8 tensors")
+        B, H, N, half = data.shape
+        d = 2 * half
+        if tuple(scale.shape) != (B, H, N, d // 16):
+            raise ValueError("scale must be [B, H, N, d/16]")
+        self.shape = (B, H, N, d)
+        self.data = data.contiguous().cuda()
+        n = scale.numel()
+        buf = torch.zeros((n + 15) // 16 * 16, dtype=torch.uint8, device=self.data.device)
+        buf[:n].copy_(scale.reshape(-1))
+        self._scale_buf = buf
+        self.scale = buf[:n].view(B, H, N, d // 16)
+        self.global_scale = float(global_scale)
+
+    def c(self) -> Nvfp4:
+        return Nvfp4(ctypes.c_void_p(self.data.data_ptr()), ctypes.c_void_p(self.scale.data_ptr()), self.global_scale)
+
+
+def prefill_nvfp4(q: Nvfp4Tensor, k: Nvfp4Tensor, v: Nvfp4Tensor, grid: Sequence[int], block_frames: int,
+                  rope_split: Sequence[int], theta: float = 1e4, eps: float = 1e-6,
+                  state: Optional[BlockState] = None, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """prefill() on NVFP4 q, k, v; the output is bf16 [B, H, N, d]."""
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k and v must share a shape")
+    B, H, N, d = q.shape
+    T, Hg, Wg = (int(x) for x in grid)
+    if N != T * Hg * Wg:
+        raise ValueError(f"N={N} but T*Hg*Wg={T * Hg * Wg}")
+    g = _geom(T, Hg, Wg, block_frames, rope_split, theta, eps)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.data.device)
+    need = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.data.device)
+    qc, kc, vc = q.c(), k.c(), v.c()
+    _check(lib.blin_prefill_nvfp4(ctypes.byref(qc), ctypes.byref(kc), ctypes.byref(vc), ctypes.c_void_p(out.data_ptr()),
+                                  B, H, d, ctypes.byref(g), state.handle if state is not None else None,
+                                  ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)))
+    return out
+
+
+def block_step_nvfp4(q: Nvfp4Tensor, k: Nvfp4Tensor, v: Nvfp4Tensor, Hg: int, Wg: int, frames: int,
+                     rope_split: Sequence[int], state: BlockState, theta: float = 1e4, eps: float = 1e-6,
+                     commit: bool = True, out: Optional[torch.Tensor] = None, stream=None,
+                     block_frames: Optional[int] = None) -> torch.Tensor:
+    """block_step() on NVFP4 q, k, v; the output is bf16."""
+    B, H, N, d = q.shape
+    if N != frames * Hg * Wg:
+        raise ValueError(f"N={N} but frames*Hg*Wg={frames * Hg * Wg}")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.data.device)
+    g = _geom(frames, Hg, Wg, frames if block_frames is None else block_frames, rope_split, theta, eps)
+    qc, kc, vc = q.c(), k.c(), v.c()
+    _check(lib.blin_block_step_nvfp4(ctypes.byref(qc), ctypes.byref(kc), ctypes.byref(vc),
+                                     ctypes.c_void_p(out.data_ptr()), B, H, d, ctypes.byref(g), state.handle,
+                                     1 if commit else 0, _stream(stream)))
     return out

@@ -260,6 +260,27 @@ static bool make_map4(CUtensorMap *m, const void *base, const Layout &l, int B, 
     return r == CUDA_SUCCESS;
 }
 
+// 4D view of NVFP4 packed data [B][H][N][d/2] bytes (contiguous): `box_rows`
+// tokens per box, no swizzle.  Tokens past N read as zeros.
+static bool make_map4_fp4(CUtensorMap *m, const void *base, int B, int H, int N, int d, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t rowb = (cuuint64_t)d / 2;
+    cuuint64_t dims[4] = {rowb, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[3] = {rowb, rowb * N, rowb * N * H};
+    cuuint32_t box[4] = {(cuuint32_t)rowb, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// NVFP4 operands of one call (NULL: bf16 / fp32 operands).
+struct Fp4In {
+    const blin_nvfp4 *q, *k, *v;
+};
+
 // ---------------------------------------------------------------- launch sequence
 static thread_local cudaEvent_t const *g_timing = nullptr;
 
@@ -275,7 +296,7 @@ static void mark(int i, bool after, cudaStream_t s) {
 // Enqueues the call.
 static blin_status run(Plan &p, const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                        const float *S_in, const float *z_in, float *S_out, float *z_out, double theta,
-                       cudaStream_t s) {
+                       cudaStream_t s, const Fp4In *fp4 = nullptr) {
     p.g.S_in = S_in;
     p.g.z_in = z_in;
     p.g.theta = theta;
@@ -290,15 +311,30 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
         CUtensorMap mq, mk, mv;
         int sk = 0, sv = 0;
         const int B = g.BH / g.H;
-        // pass 2 lands Q in spans of tiles (one box each: 256 rows at d = 32, 128 at d = 64)
-        if (!make_map4(&mq, q, g.lq, B, g.H, g.N, d, d == 32 ? 2 * kTile : kTile, &g.swap_q) ||
-            !make_map4(&mk, k, g.lq, B, g.H, g.N, d, kTile, &sk) || !make_map4(&mv, v, g.lq, B, g.H, g.N, d, kTile, &sv))
+        bool maps;
+        if (fp4) {
+            g.swap_q = 0;
+            g.sq_scale = static_cast<const uint8_t *>(fp4->q->scale);
+            g.sk_scale = static_cast<const uint8_t *>(fp4->k->scale);
+            g.sv_scale = static_cast<const uint8_t *>(fp4->v->scale);
+            g.gq = fp4->q->global_scale;
+            g.gk = fp4->k->global_scale;
+            g.gv = fp4->v->global_scale;
+            maps = make_map4_fp4(&mq, q, B, g.H, g.N, d, kTile) && make_map4_fp4(&mk, k, B, g.H, g.N, d, kTile) &&
+                   make_map4_fp4(&mv, v, B, g.H, g.N, d, kTile);
+        } else {
+            // pass 2 lands Q in spans of tiles (one box each: 256 rows at d = 32, 128 at d = 64)
+            maps = make_map4(&mq, q, g.lq, B, g.H, g.N, d, d == 32 ? 2 * kTile : kTile, &g.swap_q) &&
+                   make_map4(&mk, k, g.lq, B, g.H, g.N, d, kTile, &sk) && make_map4(&mv, v, g.lq, B, g.H, g.N, d, kTile, &sv);
+        }
+        if (!maps)
             return fail(BLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or strides rejected)");
         // both kernels hand out their work through counters that start at zero
         if ((e = cudaMemsetAsync(g.ctl, 0, 4 * sizeof(unsigned int), s)) != cudaSuccess)
             return cuda_fail(e, "work counter reset");
         mark(1, false, s);
-        if ((e = launch_partial_tc(g, d, mk, mv, s)) != cudaSuccess) return cuda_fail(e, "partial-state launch");
+        if ((e = launch_partial_tc(g, d, fp4 != nullptr, mk, mv, s)) != cudaSuccess)
+            return cuda_fail(e, "partial-state launch");
         g_launches.fetch_add(1, std::memory_order_relaxed);
         mark(1, true, s);
         mark(2, false, s);
@@ -306,7 +342,7 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
         g_launches.fetch_add(1, std::memory_order_relaxed);
         mark(2, true, s);
         mark(3, false, s);
-        if ((e = launch_output_tc(g, d, mq, o, s)) != cudaSuccess) return cuda_fail(e, "output launch");
+        if ((e = launch_output_tc(g, d, fp4 != nullptr, mq, o, s)) != cudaSuccess) return cuda_fail(e, "output launch");
         g_launches.fetch_add(1, std::memory_order_relaxed);
         mark(3, true, s);
         return BLIN_OK;
@@ -536,7 +572,8 @@ size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom *g) {
 
 static blin_status prefill_impl(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B, int H,
                                 int d, const blin_geom *g, const blin_layout *lqkv, const blin_layout *lout,
-                                blin_state *st, void *workspace, size_t ws_bytes, blin_stream stream) {
+                                blin_state *st, void *workspace, size_t ws_bytes, blin_stream stream,
+                                const Fp4In *fp4 = nullptr) {
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;
@@ -561,11 +598,14 @@ static blin_status prefill_impl(const void *q, const void *k, const void *v, voi
     if ((long long)t0 + g->T >= (1LL << 30)) return fail(BLIN_ERR_SHAPE, "frame index overflow");
     const bool tc = dt == BLIN_BF16 && tc_supported(d, g->rope_split);
     Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, t0, false, g->rope_split, g->eps, tc);
+    if (fp4 && !p.tc)
+        return fail(BLIN_ERR_SHAPE, "NVFP4 inputs need the tensor-core path (rope split (8,12,12) at d=32 or "
+                                    "(16,24,24) at d=64, and a RoPE table that fits shared memory)");
     p.g.lq = lq;
     p.g.lo = lo;
     plan_bind(p, workspace);
     rc = run(p, q, k, v, o, dt, st ? st->S : nullptr, st ? st->z : nullptr, st ? st->S : nullptr,
-             st ? st->z : nullptr, (double)g->theta, static_cast<cudaStream_t>(stream));
+             st ? st->z : nullptr, (double)g->theta, static_cast<cudaStream_t>(stream), fp4);
     if (rc != BLIN_OK) return rc;
     if (st) {
         if ((rc = mark_state_use(st, static_cast<cudaStream_t>(stream))) != BLIN_OK) return rc;
@@ -576,7 +616,8 @@ static blin_status prefill_impl(const void *q, const void *k, const void *v, voi
 
 static blin_status block_step_impl(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B,
                                    int H, int d, const blin_geom *g, const blin_layout *lqkv,
-                                   const blin_layout *lout, blin_state *st, int commit, blin_stream stream) {
+                                   const blin_layout *lout, blin_state *st, int commit, blin_stream stream,
+                                   const Fp4In *fp4 = nullptr) {
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;
@@ -602,12 +643,15 @@ static blin_status block_step_impl(const void *q, const void *k, const void *v, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool tc = dt == BLIN_BF16 && tc_supported(d, g->rope_split);
     Plan p = make_plan(B, H, d, frames, g->Hgt, g->Wid, frames, st->t_next, true, g->rope_split, g->eps, tc);
+    if (fp4 && !p.tc)
+        return fail(BLIN_ERR_SHAPE, "NVFP4 inputs need the tensor-core path (rope split (8,12,12) at d=32 or "
+                                    "(16,24,24) at d=64, and a RoPE table that fits shared memory)");
     p.g.lq = lq;
     p.g.lo = lo;
     if ((rc = ensure_scratch(st, plan_bytes(p), s)) != BLIN_OK) return rc;
     plan_bind(p, st->scratch);
     rc = run(p, q, k, v, o, dt, st->S, st->z, commit ? st->S : nullptr, commit ? st->z : nullptr,
-             (double)g->theta, s);
+             (double)g->theta, s, fp4);
     if (rc != BLIN_OK) return rc;
     if ((rc = mark_state_use(st, s)) != BLIN_OK) return rc;
     if (commit) st->t_next += frames;
@@ -624,6 +668,38 @@ blin_status blin_prefill_strided(const void *q, const void *k, const void *v, vo
                                  const blin_layout *o_layout, blin_state *st, void *workspace, size_t ws_bytes,
                                  blin_stream stream) {
     return prefill_impl(q, k, v, o, dt, B, H, d, g, qkv_layout, o_layout, st, workspace, ws_bytes, stream);
+}
+
+// NVFP4 operand checks: data and scale 16-byte aligned, positive finite global scale.
+static blin_status check_fp4(const blin_nvfp4 *x, const char *name) {
+    if (x == nullptr || x->data == nullptr || x->scale == nullptr)
+        return fail(BLIN_ERR_INVALID_ARG, "NVFP4 %s: operand, data and scale must be non-NULL", name);
+    if (!aligned16(x->data) || !aligned16(x->scale))
+        return fail(BLIN_ERR_ALIGN, "NVFP4 %s: data and scale must be 16-byte aligned", name);
+    if (!(x->global_scale > 0.f) || !std::isfinite(x->global_scale))
+        return fail(BLIN_ERR_INVALID_ARG, "NVFP4 %s: global scale must be finite and > 0", name);
+    return BLIN_OK;
+}
+
+blin_status blin_prefill_nvfp4(const blin_nvfp4 *q, const blin_nvfp4 *k, const blin_nvfp4 *v, void *o, int B, int H,
+                               int d, const blin_geom *g, blin_state *st, void *workspace, size_t ws_bytes,
+                               blin_stream stream) {
+    blin_status rc;
+    if ((rc = check_fp4(q, "q")) != BLIN_OK || (rc = check_fp4(k, "k")) != BLIN_OK || (rc = check_fp4(v, "v")) != BLIN_OK)
+        return rc;
+    const Fp4In fp4{q, k, v};
+    return prefill_impl(q->data, k->data, v->data, o, BLIN_BF16, B, H, d, g, nullptr, nullptr, st, workspace, ws_bytes,
+                        stream, &fp4);
+}
+
+blin_status blin_block_step_nvfp4(const blin_nvfp4 *q, const blin_nvfp4 *k, const blin_nvfp4 *v, void *o, int B,
+                                  int H, int d, const blin_geom *g, blin_state *st, int commit, blin_stream stream) {
+    blin_status rc;
+    if ((rc = check_fp4(q, "q")) != BLIN_OK || (rc = check_fp4(k, "k")) != BLIN_OK || (rc = check_fp4(v, "v")) != BLIN_OK)
+        return rc;
+    const Fp4In fp4{q, k, v};
+    return block_step_impl(q->data, k->data, v->data, o, BLIN_BF16, B, H, d, g, nullptr, nullptr, st, commit, stream,
+                           &fp4);
 }
 
 blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt, int B, int H,

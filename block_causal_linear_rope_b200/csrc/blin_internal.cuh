@@ -48,6 +48,9 @@ struct KGeom {
     float *S_out, *z_out;      // cache after the call (NULL: not written)
     Layout lq, lo;             // element strides of q, k, v (shared) and of o
     int swap_q;                // 1: the q/k/v tensor maps order the head dimension before the token one
+    // NVFP4 inputs: scale bytes [B*H*N][d/16] of q, k, v and the tensors' global scales
+    const uint8_t *sq_scale, *sk_scale, *sv_scale;
+    float gq, gk, gv;
     // ---- work units: every block is split into state chunks (pass 1) and, on the
     // tensor-core path, query groups (pass 2) of whole tiles; the first, middle and
     // last blocks of a call may differ in length.
@@ -104,8 +107,11 @@ cudaError_t launch_output_simt(const KGeom &g, int d, bool bf16, const void *q, 
 // q/k/v as 4D [B][H][N][d] with the call's strides.
 bool tc_supported(int d, const int split[3]);
 int tc_table_smem_limit(int d);
-cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv, cudaStream_t s);
-cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, void *o, cudaStream_t s);
+// `fp4`: NVFP4 inputs (packed E2M1 data through the maps, scales and global
+// scales through the geometry).
+cudaError_t launch_partial_tc(const KGeom &g, int d, bool fp4, const CUtensorMap &mk, const CUtensorMap &mv,
+                              cudaStream_t s);
+cudaError_t launch_output_tc(const KGeom &g, int d, bool fp4, const CUtensorMap &mq, void *o, cudaStream_t s);
 
 // Device watchdog access.
 cudaError_t read_and_clear_watchdog(int *code);

@@ -118,7 +118,10 @@ static cudaError_t set_smem(int bytes) {
 // Largest RoPE table (bytes) the tensor-core kernels can hold in shared memory
 // next to their rings (227 KB per CTA).
 int tc_table_smem_limit(int d) {
-    const int fixed = d == 32 ? std::max(K1Cfg<32>::FIXED, K2Cfg<32>::FIXED) : std::max(K1Cfg<64>::FIXED, K2Cfg<64>::FIXED);
+    const int fixed = d == 32 ? std::max(std::max(K1Cfg<32>::FIXED, K2Cfg<32>::FIXED),
+                                         std::max(K1Cfg<32, true>::FIXED, K2Cfg<32, true>::FIXED))
+                              : std::max(std::max(K1Cfg<64>::FIXED, K2Cfg<64>::FIXED),
+                                         std::max(K1Cfg<64, true>::FIXED, K2Cfg<64, true>::FIXED));
     return std::min(24 * 1024, 227 * 1024 - fixed);
 }
 
@@ -170,29 +173,38 @@ static cudaError_t launch_persistent(bool pdl, int smem, int threads, long long 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_partial_tc(const KGeom &g, int d, const CUtensorMap &mk, const CUtensorMap &mv, cudaStream_t s) {
-    int *wd = watchdog_ptr();
-    if (wd == nullptr) return cudaErrorInvalidDevice;
+template <int D, int PT, int PY, int PX, bool FP4>
+static cudaError_t partial_tc(const KGeom &g, const CUtensorMap &mk, const CUtensorMap &mv, int *wd, cudaStream_t s) {
+    using C = K1Cfg<D, FP4>;
     const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
-    const long long units = (long long)g.BH * g.U1;
-    if (d == 32)
-        return launch_persistent<partial_tc_kernel<32, 4, 6, 6>>(false, K1Cfg<32>::FIXED + tab, K1Cfg<32>::THREADS, units,
-                                                                 K1Cfg<32>::NP, s, mk, mv, g, wd);
-    return launch_persistent<partial_tc_kernel<64, 8, 12, 12>>(false, K1Cfg<64>::FIXED + tab, K1Cfg<64>::THREADS, units,
-                                                               K1Cfg<64>::NP, s, mk, mv, g, wd);
+    return launch_persistent<partial_tc_kernel<D, PT, PY, PX, FP4>>(false, C::FIXED + tab, C::THREADS,
+                                                                     (long long)g.BH * g.U1, C::NP, s, mk, mv, g, wd);
 }
 
-cudaError_t launch_output_tc(const KGeom &g, int d, const CUtensorMap &mq, void *o, cudaStream_t s) {
+template <int D, int PT, int PY, int PX, bool FP4>
+static cudaError_t output_tc(const KGeom &g, const CUtensorMap &mq, __nv_bfloat16 *o, int *wd, cudaStream_t s) {
+    using C = K2Cfg<D, FP4>;
+    const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
+    return launch_persistent<output_tc_kernel<D, PT, PY, PX, FP4>>(true, C::FIXED + tab, C::THREADS,
+                                                                    (long long)g.BH * g.U2, C::NP, s, mq, g, o, wd);
+}
+
+cudaError_t launch_partial_tc(const KGeom &g, int d, bool fp4, const CUtensorMap &mk, const CUtensorMap &mv,
+                              cudaStream_t s) {
     int *wd = watchdog_ptr();
     if (wd == nullptr) return cudaErrorInvalidDevice;
-    const int tab = g.tab_smem ? g.tab_smem_bytes : 0;
-    const long long units = (long long)g.BH * g.U2;
+    if (d == 32)
+        return fp4 ? partial_tc<32, 4, 6, 6, true>(g, mk, mv, wd, s) : partial_tc<32, 4, 6, 6, false>(g, mk, mv, wd, s);
+    return fp4 ? partial_tc<64, 8, 12, 12, true>(g, mk, mv, wd, s) : partial_tc<64, 8, 12, 12, false>(g, mk, mv, wd, s);
+}
+
+cudaError_t launch_output_tc(const KGeom &g, int d, bool fp4, const CUtensorMap &mq, void *o, cudaStream_t s) {
+    int *wd = watchdog_ptr();
+    if (wd == nullptr) return cudaErrorInvalidDevice;
     __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
     if (d == 32)
-        return launch_persistent<output_tc_kernel<32, 4, 6, 6>>(true, K2Cfg<32>::FIXED + tab, K2Cfg<32>::THREADS, units,
-                                                                K2Cfg<32>::NP, s, mq, g, ob, wd);
-    return launch_persistent<output_tc_kernel<64, 8, 12, 12>>(true, K2Cfg<64>::FIXED + tab, K2Cfg<64>::THREADS, units,
-                                                              K2Cfg<64>::NP, s, mq, g, ob, wd);
+        return fp4 ? output_tc<32, 4, 6, 6, true>(g, mq, ob, wd, s) : output_tc<32, 4, 6, 6, false>(g, mq, ob, wd, s);
+    return fp4 ? output_tc<64, 8, 12, 12, true>(g, mq, ob, wd, s) : output_tc<64, 8, 12, 12, false>(g, mq, ob, wd, s);
 }
 
 }  // namespace blin

@@ -284,53 +284,142 @@ struct TcCfg {
     static constexpr int E = D * D + D, E4 = E / 4;
     // control block: [NP][BARS_PER_PIPE] mbarriers, 16 B of flags, [NP][INFO_PER_PIPE] record ints
     static constexpr int BARS_PER_PIPE = 64;
-    static constexpr int INFO_PER_PIPE = 128;
+    static constexpr int INFO_PER_PIPE = 160;
     static constexpr int OFF_FLAGS = NP * BARS_PER_PIPE * 8;
     static constexpr int OFF_INFO = OFF_FLAGS + 16;
     static constexpr int CTRL = (OFF_INFO + NP * INFO_PER_PIPE * 4 + 1023) / 1024 * 1024;
     static_assert(NP * NA * ACOLS <= (int)TCOLS, "TMEM columns");
 };
 
+// NVFP4 inputs (FP4 = true): a tile of 128 tokens is d/2 packed bytes per token
+// (two E2M1 codes a byte) and d/16 E4M3 scale bytes per token.
 template <int D>
+struct Fp4Tile {
+    static constexpr int DB = D / 2 * kTile;        // packed data bytes of one tile
+    static constexpr int S1 = D / 16;               // scale bytes per token
+    static constexpr int SB = S1 * kTile + 32;      // scale bytes of one tile, with room to round the copy to 16 B
+    static constexpr int TABS = 256 * 4 + 256 * 2;  // dequantisation tables: code pairs, E4M3 scales
+};
+
+template <int D, bool FP4 = false>
 struct K1Cfg : TcCfg<D> {
     using B = TcCfg<D>;
+    using F = Fp4Tile<D>;
     static constexpr int M1 = D == 32 ? 64 : 128;          // [K~^T ; phi(K)^T]
     static constexpr int N1 = D == 32 ? D + 8 : D + 16;    // [V | ones]
-    static constexpr int NK = D == 32 ? 4 : 3;             // K landing slots (free once read)
-    static constexpr int NV = 4;                           // V landing slots (free once the MMA is done)
-    static constexpr int PIPE = (NK + NV + 2 * B::NO) * B::TB;
-    static constexpr int OFF_ONES = B::NP * PIPE;          // above every V slot: positive LBO
+    // landing slots: bf16 -- one K tile (free once read); NVFP4 -- a tile's K and V data
+    // and scales (free once read: V is dequantised into the operand slot)
+    static constexpr int LSLOT = FP4 ? (2 * (F::DB + F::SB) + 1023) / 1024 * 1024 : B::TB;
+    static constexpr int NK = FP4 ? (D == 32 ? 8 : 6) : (D == 32 ? 4 : 3);
+    static constexpr int NV = FP4 ? 0 : 4;                 // bf16 V landing slots (read in place by the MMA)
+    static constexpr int NTD = FP4 ? 4 : NV;               // tile-done barriers
+    static constexpr int OPND = (FP4 ? 3 : 2) * B::TB;     // operand slot: K~ | phi (| dequantised V)
+    static constexpr int PIPE = NK * LSLOT + NV * B::TB + B::NO * OPND;
+    static constexpr int OFF_ONES = B::NP * PIPE;          // above every V tile: positive LBO
     static constexpr int OFF_CTRL = OFF_ONES + B::TB;
-    static constexpr int FIXED = OFF_CTRL + B::CTRL + 1024;  // + alignment slack; the RoPE table follows
-    static constexpr int NBAR = 2 * NK + NV + B::NO + 2 * B::NA + 2 * B::NINFO + 1;
-    static constexpr int NINF = 5 * NK + 4 * B::NO + B::NINFO;
+    static constexpr int TABS = FP4 ? F::TABS : 0;         // after the control block
+    static constexpr int FIXED = OFF_CTRL + B::CTRL + TABS + 1024;  // + alignment slack; the RoPE table follows
+    static constexpr int LREC = 7;                         // ints per landing record
+    static constexpr int NBAR = 2 * NK + NTD + B::NO + 2 * B::NA + 2 * B::NINFO + 1;
+    static constexpr int NINF = LREC * NK + 4 * B::NO + B::NINFO;
     static_assert(NBAR <= B::BARS_PER_PIPE && NINF <= B::INFO_PER_PIPE, "control block");
-    static_assert(NV > B::NO, "an operand slot's release is read from the V ring's tile-done barriers");
+    static_assert(NTD > B::NO, "an operand slot's release is read from the tile-done barriers");
     static_assert(OFF_ONES < (1 << 18), "LBO field range");
     static_assert(PIPE % 1024 == 0, "pipelines keep 1024-byte alignment");
 };
 
-template <int D>
+template <int D, bool FP4 = false>
 struct K2Cfg : TcCfg<D> {
     using B = TcCfg<D>;
-    // Q lands in slots of SPAN consecutive tiles, one TMA box each: the copy engine moves
-    // a 16-KB box in about the time of an 8-KB one, so fewer, larger boxes move more bytes
-    static constexpr int SPAN = D == 32 ? 2 : 1;           // tiles per Q landing slot
-    static constexpr int NLS = 3;                          // Q landing slots
-    static constexpr int NL = NLS * SPAN;                  // Q tiles in the landing ring
+    using F = Fp4Tile<D>;
+    // bf16 Q lands in slots of SPAN consecutive tiles, one TMA box each (fewer, larger
+    // boxes); NVFP4 Q in slots of one tile's data and scales
+    static constexpr int SPAN = FP4 ? 1 : (D == 32 ? 2 : 1);  // tiles per Q landing slot
+    static constexpr int NLS = FP4 ? 8 : 3;                    // Q landing slots
+    static constexpr int LSLOT = FP4 ? (F::DB + F::SB + 1023) / 1024 * 1024 : SPAN * B::TB;
+    static constexpr int NL = NLS * SPAN;                      // Q tiles in the landing ring
     static constexpr int NT = B::NA > B::NO + 1 ? B::NA : B::NO + 1;  // tile-done barriers
     static constexpr int N2 = OutB<D>::N;
     static constexpr int BATOM = OutB<D>::BATOM;
     static constexpr int IMG = OutB<D>::IMG;
     static constexpr int PRE = (D * D + D) * 4;            // one fp32 prefix state (S, z)
     // Q ring, operand ring, O staging (4 warps x 32 rows), 2 B images, prefix state
-    static constexpr int PIPE = (NL * B::TB + B::NO * 2 * B::TB + B::TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
+    static constexpr int PIPE = (NLS * LSLOT + B::NO * 2 * B::TB + B::TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
     static constexpr int OFF_CTRL = B::NP * PIPE;
-    static constexpr int FIXED = OFF_CTRL + B::CTRL + 1024;
+    static constexpr int TABS = FP4 ? F::TABS : 0;
+    static constexpr int FIXED = OFF_CTRL + B::CTRL + TABS + 1024;
     static constexpr int NBAR = 2 * NLS + B::NO + NT + B::NA + 4 + 2 * B::NINFO + 1;
     static constexpr int NINF = 8 * NLS + 6 * B::NO + 4 * B::NINFO;
     static_assert(NBAR <= B::BARS_PER_PIPE && NINF <= B::INFO_PER_PIPE, "control block");
 };
+
+// ---------------------------------------------------------------------------- NVFP4 decoding
+// Tables in shared memory, filled once per CTA: pair[byte] = the two E2M1 values of a
+// packed byte as bf16x2 (even element in the low half); e4m3[byte] = the E4M3 scale as
+// bf16 bits.  Every E2M1 x E4M3 product has at most 6 significant bits, so multiplying
+// the bf16 pair by the bf16 scale is exact: the tile's bf16 values are exactly the
+// NVFP4 values up to the tensor's global scale (applied in fp32 by the epilogues).
+__device__ __forceinline__ float e2m1_value(int c) {
+    const int e = (c >> 1) & 3, m = c & 1;
+    const float mag = e == 0 ? 0.5f * m : ldexpf(1.0f + 0.5f * m, e - 1);
+    return (c & 8) ? -mag : mag;
+}
+__device__ __forceinline__ float e4m3_value(int c) {
+    const int e = (c >> 3) & 15, m = c & 7;
+    const float mag = e == 0 ? ldexpf(m / 8.0f, -6) : ldexpf(1.0f + m / 8.0f, e - 7);
+    return (c & 0x80) ? -mag : mag;  // codes 0x7f / 0xff (NaN) are never produced by a valid encoder
+}
+__device__ __forceinline__ void fill_fp4_tables(uint8_t *tabs, int tid, int nthreads) {
+    uint32_t *pair = reinterpret_cast<uint32_t *>(tabs);
+    uint16_t *sc = reinterpret_cast<uint16_t *>(tabs + 1024);
+    for (int i = tid; i < 256; i += nthreads) {
+        pair[i] = pack_bf16x2(e2m1_value(i & 15), e2m1_value(i >> 4));
+        const __nv_bfloat16 h = __float2bfloat16_rn(e4m3_value(i));
+        sc[i] = *reinterpret_cast<const uint16_t *>(&h);
+    }
+}
+// One token row: d/2 packed bytes at `data`, d/16 scale bytes at `scale` -> bf16x2 words.
+template <int D>
+__device__ __forceinline__ void fp4_row(const uint8_t *data, const uint8_t *scale, const uint8_t *tabs,
+                                        uint32_t (&w)[D / 2]) {
+    const uint32_t *pair = reinterpret_cast<const uint32_t *>(tabs);
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(tabs + 1024);
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {  // 16 bytes = 32 elements = two scale blocks
+        const uint4 v = *reinterpret_cast<const uint4 *>(data + 16 * j);
+        const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t sbits = sc[scale[2 * j + half]];
+            const uint32_t s2 = sbits | (sbits << 16);
+            const __nv_bfloat162 s2h = *reinterpret_cast<const __nv_bfloat162 *>(&s2);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int byte_i = 8 * half + q;
+                const uint32_t byte = (words[byte_i >> 2] >> (8 * (byte_i & 3))) & 0xFFu;
+                const uint32_t pv = pair[byte];
+                const __nv_bfloat162 prod = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&pv), s2h);
+                w[16 * j + byte_i] = *reinterpret_cast<const uint32_t *>(&prod);
+            }
+        }
+    }
+}
+// Bytes [a0, a1) of a tile's scale rows: `rows` tokens from global token row `row0`
+// (of `total` rows), rounded outwards to 16 bytes (the allocation is padded to 16 B).
+struct ScaleSpan {
+    long long a0;
+    int bytes, off;
+};
+template <int D>
+__device__ __forceinline__ ScaleSpan scale_span(long long row0, int rows, long long total) {
+    constexpr int S1 = D / 16;
+    const long long b0 = row0 * S1, e = min(row0 + rows, total) * S1;
+    ScaleSpan sp;
+    sp.a0 = b0 & ~15LL;
+    sp.bytes = (int)(((e + 15) & ~15LL) - sp.a0);
+    sp.off = (int)(b0 - sp.a0);
+    return sp;
+}
 
 // Named barrier of all transform warps of a CTA (the RoPE table fill, before
 // any work starts; every other hand-over is an mbarrier with a bounded wait).
@@ -346,44 +435,51 @@ struct PipeSmem {
 };
 
 // ---------------------------------------------------------------------------- pass-1 pipeline
-template <int D, int PT, int PY, int PX>
+template <int D, int PT, int PY, int PX, bool FP4>
 struct Pass1 {
-    using C = K1Cfg<D>;
-    static constexpr int NK = C::NK, NV = C::NV, NO = C::NO, NA = C::NA, TB = C::TB, ROWB = C::ROWB, E = C::E;
+    using C = K1Cfg<D, FP4>;
+    using F = Fp4Tile<D>;
+    static constexpr int NK = C::NK, NV = C::NV, NTD = C::NTD, NO = C::NO, NA = C::NA, TB = C::TB, ROWB = C::ROWB,
+                         E = C::E, LREC = C::LREC;
+    static constexpr int NVD = NV > 0 ? NV : 1;  // divisor for the bf16 V ring (unused with NVFP4)
     const KGeom &g;
     PipeSmem ps;
     int *wd;
     uint8_t *kring, *vring, *opnd;
+    const uint8_t *tabs;  // NVFP4 decoding tables
     int *linfo, *oinfo, *cinfo;
     uint32_t tmem;
 
-    __device__ Pass1(const KGeom &g_, const PipeSmem &ps_, int *wd_, uint32_t tmem_base) : g(g_), ps(ps_), wd(wd_) {
+    __device__ Pass1(const KGeom &g_, const PipeSmem &ps_, int *wd_, uint32_t tmem_base, const uint8_t *tabs_)
+        : g(g_), ps(ps_), wd(wd_), tabs(tabs_) {
         kring = ps.base;
-        vring = kring + NK * TB;
+        vring = kring + NK * C::LSLOT;
         opnd = vring + NV * TB;
         linfo = ps.info;
-        oinfo = linfo + 5 * NK;
+        oinfo = linfo + LREC * NK;
         cinfo = oinfo + 4 * NO;
         tmem = tmem_base;
     }
-    __device__ uint8_t *lk(int s) const { return kring + s * TB; }
+    __device__ uint8_t *lk(int s) const { return kring + s * C::LSLOT; }
     __device__ uint8_t *lv(int s) const { return vring + s * TB; }
-    __device__ uint8_t *ok_(int s) const { return opnd + s * 2 * TB; }
-    __device__ uint8_t *op_(int s) const { return opnd + s * 2 * TB + TB; }
-    // kfull[s]: K and V of the tile in K slot s have landed; kempty[s]: its K is read (4 warps);
-    // tdone[s]: the tile in V slot s is multiplied (V slot and its operand slot free);
+    __device__ uint8_t *ok_(int s) const { return opnd + s * C::OPND; }
+    __device__ uint8_t *op_(int s) const { return opnd + s * C::OPND + TB; }
+    __device__ uint8_t *ov_(int s) const { return opnd + s * C::OPND + 2 * TB; }  // NVFP4: dequantised V
+    // kfull[s]: the tile in landing slot s has landed (bf16: K, and V in its V slot; NVFP4:
+    // K and V data and scales); kempty[s]: slot s is read (4 warps); tdone[s]: the tile
+    // k = s (mod NTD) is multiplied (its operand slot, and bf16 V slot, are free);
     // ofull[s]: operand slot s written (4 warps); accf/acce: chunk accumulator ready / read;
     // cfull/cempty: chunk record ring (producer -> epilogue)
     __device__ uint32_t bar(int i) const { return ptx::smem_u32(ps.bars + i); }
     __device__ uint32_t kfull(int s) const { return bar(s); }
     __device__ uint32_t kempty(int s) const { return bar(NK + s); }
     __device__ uint32_t tdone(int s) const { return bar(2 * NK + s); }
-    __device__ uint32_t ofull(int s) const { return bar(2 * NK + NV + s); }
-    __device__ uint32_t accf(int a) const { return bar(2 * NK + NV + NO + a); }
-    __device__ uint32_t acce(int a) const { return bar(2 * NK + NV + NO + NA + a); }
-    __device__ uint32_t cfull(int i) const { return bar(2 * NK + NV + NO + 2 * NA + i); }
-    __device__ uint32_t cempty(int i) const { return bar(2 * NK + NV + NO + 2 * NA + C::NINFO + i); }
-    __device__ uint32_t drain() const { return bar(2 * NK + NV + NO + 2 * NA + 2 * C::NINFO); }
+    __device__ uint32_t ofull(int s) const { return bar(2 * NK + NTD + s); }
+    __device__ uint32_t accf(int a) const { return bar(2 * NK + NTD + NO + a); }
+    __device__ uint32_t acce(int a) const { return bar(2 * NK + NTD + NO + NA + a); }
+    __device__ uint32_t cfull(int i) const { return bar(2 * NK + NTD + NO + 2 * NA + i); }
+    __device__ uint32_t cempty(int i) const { return bar(2 * NK + NTD + NO + 2 * NA + C::NINFO + i); }
+    __device__ uint32_t drain() const { return bar(2 * NK + NTD + NO + 2 * NA + 2 * C::NINFO); }
 
     __device__ static void init_barriers(uint64_t *b) {
         auto at = [&](int i) { return ptx::smem_u32(b + i); };
@@ -391,17 +487,17 @@ struct Pass1 {
             ptx::mbar_init(at(s), 1);       // kfull: producer (+ TMA bytes)
             ptx::mbar_init(at(NK + s), 4);  // kempty: transform warps
         }
-        for (int s = 0; s < NV; ++s) ptx::mbar_init(at(2 * NK + s), 1);       // tdone: commit
-        for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NK + NV + s), 4);  // ofull
+        for (int s = 0; s < NTD; ++s) ptx::mbar_init(at(2 * NK + s), 1);       // tdone: commit
+        for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NK + NTD + s), 4);  // ofull
         for (int a = 0; a < NA; ++a) {
-            ptx::mbar_init(at(2 * NK + NV + NO + a), 1);       // accf: commit
-            ptx::mbar_init(at(2 * NK + NV + NO + NA + a), 4);  // acce: epilogue warps
+            ptx::mbar_init(at(2 * NK + NTD + NO + a), 1);       // accf: commit
+            ptx::mbar_init(at(2 * NK + NTD + NO + NA + a), 4);  // acce: epilogue warps
         }
         for (int i = 0; i < C::NINFO; ++i) {
-            ptx::mbar_init(at(2 * NK + NV + NO + 2 * NA + i), 1);            // cfull: producer
-            ptx::mbar_init(at(2 * NK + NV + NO + 2 * NA + C::NINFO + i), 4);  // cempty: epilogue
+            ptx::mbar_init(at(2 * NK + NTD + NO + 2 * NA + i), 1);            // cfull: producer
+            ptx::mbar_init(at(2 * NK + NTD + NO + 2 * NA + C::NINFO + i), 4);  // cempty: epilogue
         }
-        ptx::mbar_init(at(2 * NK + NV + NO + 2 * NA + 2 * C::NINFO), 1);  // drain
+        ptx::mbar_init(at(2 * NK + NTD + NO + 2 * NA + 2 * C::NINFO), 1);  // drain
     }
 
     __device__ int nc_of(int b) const { return units_of_block(g, b, g.nc_first, g.nc_mid, g.nc_last); }
@@ -450,28 +546,42 @@ struct Pass1 {
             if (!ok) break;
             ++j;
             for (int t = t_lo; t < t_hi; ++t, ++k) {
-                const int sk = k % NK, sv = k % NV;
+                const int sk = k % NK, sv = k % NVD;
                 const int n = fb * g.HW + t * kTile;  // token (within the head) of the tile's first row
+                // NVFP4: this tile's scale bytes, rounded outwards to 16 B (same for K and V)
+                ScaleSpan sp{};
+                if constexpr (FP4) sp = scale_span<D>((long long)bh * g.N + n, kTile, (long long)g.BH * g.N);
                 if (lead) {
                     if ((k >= NK && !ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs)) ||
-                        (k >= NV && !ptx::mbar_wait_bounded(tdone(sv), ((k / NV) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs))) {
+                        (!FP4 && k >= NV &&
+                         !ptx::mbar_wait_bounded(tdone(sv), ((k / NVD) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs))) {
                         ok = false;
                     } else {
-                        int *inf = linfo + 5 * sk;
+                        int *inf = linfo + LREC * sk;
                         inf[0] = u;
                         inf[1] = t - t_lo;
                         inf[2] = min(kTile, L - t * kTile);
                         inf[3] = t == t_hi - 1;
                         inf[4] = n;
-                        ptx::mbar_arrive_expect_tx(kfull(sk), 2 * TB);
+                        inf[5] = sp.off;
+                        ptx::mbar_arrive_expect_tx(kfull(sk), FP4 ? 2 * (F::DB + sp.bytes) : 2 * TB);
                     }
                 }
                 // both slots are free (and the bytes expected) before either load goes out
                 ok = __shfl_sync(3u, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
                 const MapCoord mc = map_coord(n, hh, g.swap_q);
-                if (lead) ptx::tma_load_4d_hint(ptx::smem_u32(lk(sk)), mk, kfull(sk), 0, mc.y, mc.z, bb, policy);
-                else ptx::tma_load_4d_hint(ptx::smem_u32(lv(sv)), mv, kfull(sk), 0, mc.y, mc.z, bb, policy);
+                if constexpr (FP4) {
+                    // lane 0: K data and scales; lane 1: V data and scales
+                    uint8_t *slot = lk(sk);
+                    const uint8_t *sg = lead ? g.sk_scale : g.sv_scale;
+                    ptx::tma_load_4d_hint(ptx::smem_u32(slot + (lead ? 0 : F::DB)), lead ? mk : mv, kfull(sk), 0, mc.y,
+                                          mc.z, bb, policy);
+                    ptx::bulk_load(ptx::smem_u32(slot + 2 * F::DB + (lead ? 0 : F::SB)), sg + sp.a0, sp.bytes, kfull(sk));
+                } else {
+                    if (lead) ptx::tma_load_4d_hint(ptx::smem_u32(lk(sk)), mk, kfull(sk), 0, mc.y, mc.z, bb, policy);
+                    else ptx::tma_load_4d_hint(ptx::smem_u32(lv(sv)), mv, kfull(sk), 0, mc.y, mc.z, bb, policy);
+                }
             }
         }
         if (!lead) return;
@@ -479,7 +589,7 @@ struct Pass1 {
         const int sk = k % NK;
         bool marked = false;
         if (ok && (k < NK || ptx::mbar_wait_bounded(kempty(sk), ((k / NK) - 1) & 1, wd, WD_P1_EMPTY, kWaitLimitNs))) {
-            linfo[5 * sk] = kEndFirst;
+            linfo[LREC * sk] = kEndFirst;
             ptx::mbar_arrive(kfull(sk));
             marked = true;
         }
@@ -519,8 +629,8 @@ struct Pass1 {
                 break;
             }
             ptx::tc_fence_after_sync();
-            const int sv = k % NV;  // the tile's V slot (same tile order as the producer)
-            const uint32_t va = ptx::smem_u32(lv(sv));
+            // the tile's V: bf16 in place in its landing slot; NVFP4 dequantised in the operand slot
+            const uint32_t va = FP4 ? ptx::smem_u32(ov_(so)) : ptx::smem_u32(lv(k % NVD));
             // A (MN-major): M atom 0 = K~ rows, atom 1 (+TB) = phi rows; B: V | ones.
             // Consecutive K steps are 16 token rows (16 * ROWB bytes: ROWB in the address field).
             const uint64_t ad = ptx::smem_desc(ptx::smem_u32(ok_(so)), TB, 8 * ROWB, C::LAYOUT);
@@ -530,7 +640,7 @@ struct Pass1 {
             for (int kk = 0; kk < kTile / 16; ++kk)
                 ptx::mma_bf16_ss(dacc, ad + static_cast<uint64_t>(kk * ROWB), bd + static_cast<uint64_t>(kk * ROWB),
                                  IDESC, (t > 0 || kk > 0) ? 1u : 0u);
-            ptx::mma_commit(tdone(sv));
+            ptx::mma_commit(tdone(k % NTD));
             if (last) {
                 ptx::mma_commit(accf(a));
                 ++nu;
@@ -553,21 +663,29 @@ struct Pass1 {
                 ps.flags[0] = 1;
                 break;
             }
-            const int *inf = linfo + 5 * sk;
+            const int *inf = linfo + LREC * sk;
             const int u = ld_volatile(inf), t = ld_volatile(inf + 1), valid = ld_volatile(inf + 2);
             const int last = ld_volatile(inf + 3), n = ld_volatile(inf + 4);
             // read this row of K; rows past the chunk also clear their V row
             // (the MMA reads V in place: other blocks' tokens must add nothing)
-            uint32_t w[D / 2], ph[D / 2];
+            uint32_t w[D / 2], ph[D / 2], vw[D / 2];
             const bool live = u >= 0 && r < valid;
-            if (live) load_row<D>(lk(sk), r, w);
-            else if (u >= 0) zero_row<D>(lv(k % NV), r);
+            if constexpr (FP4) {
+                if (live) {
+                    const uint8_t *slot = lk(sk), *scl = slot + 2 * F::DB + ld_volatile(inf + 5) + r * F::S1;
+                    fp4_row<D>(slot + r * (D / 2), scl, tabs, w);
+                    fp4_row<D>(slot + F::DB + r * (D / 2), scl + F::SB, tabs, vw);
+                }
+            } else {
+                if (live) load_row<D>(lk(sk), r, w);
+                else if (u >= 0) zero_row<D>(lv(k % NVD), r);
+            }
             // the next TMA into this K slot writes through the async proxy: order
             // this thread's generic reads of the slot before it
             ptx::fence_proxy_async_smem();
             if (u >= 0) warp_arrive(kempty(sk), lane);
             // operand slot so was last used by tile k - NO: wait for its MMAs
-            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NV), ((k - NO) / NV) & 1, wd, WD_P1_READY,
+            if (k >= NO && !ptx::mbar_wait_bounded(tdone((k - NO) % NTD), ((k - NO) / NTD) & 1, wd, WD_P1_READY,
                                                    kWaitLimitNs)) {
                 ps.flags[0] = 1;
                 break;
@@ -583,9 +701,11 @@ struct Pass1 {
                 phi_rope_row<D, PT, PY, PX, false>(w, ph, tab, tp, nullptr);
                 store_row<D>(ok_(so), r, w);
                 store_row<D>(op_(so), r, ph);
+                if constexpr (FP4) store_row<D>(ov_(so), r, vw);
             } else {  // rows past the chunk add nothing
                 zero_row<D>(ok_(so), r);
                 zero_row<D>(op_(so), r);
+                if constexpr (FP4) zero_row<D>(ov_(so), r);
             }
             ptx::fence_proxy_async_smem();
             if (r == 0) {
@@ -628,10 +748,15 @@ struct Pass1 {
             const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
             if (sub < 2) {
                 const int m = RPS * sub + lane;  // P row
+                const float sp = FP4 ? g.gk * g.gv : 1.0f;  // NVFP4: the tensors' global scales
 #pragma unroll
                 for (int half = 0; half < D / 32; ++half) {
                     float v[32];
                     ptx::tmem_ld_32cols(taddr + 32 * half, v);
+                    if constexpr (FP4) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) v[q] *= sp;
+                    }
                     if (lane < RPS) {
                         float4 *dst = reinterpret_cast<float4 *>(out + m * D + 32 * half);
 #pragma unroll
@@ -641,6 +766,7 @@ struct Pass1 {
             } else {
                 float zv, unused;
                 tmem_ld_2cols(taddr + D, zv, unused);
+                if constexpr (FP4) zv *= g.gk;
                 if (lane < RPS) out[D * D + RPS * (sub - 2) + lane] = zv;
             }
             ptx::tc_fence_before_sync();
@@ -650,21 +776,24 @@ struct Pass1 {
 };
 
 // ---------------------------------------------------------------------------- pass-2 pipeline
-template <int D, int PT, int PY, int PX>
+template <int D, int PT, int PY, int PX, bool FP4>
 struct Pass2 {
-    using C = K2Cfg<D>;
+    using C = K2Cfg<D, FP4>;
+    using F = Fp4Tile<D>;
     static constexpr int NL = C::NL, NLS = C::NLS, SPAN = C::SPAN, NO = C::NO, NA = C::NA, NT = C::NT, TB = C::TB,
                          ROWB = C::ROWB, E = C::E;
     const KGeom &g;
     PipeSmem ps;
     int *wd;
     uint8_t *land, *opnd, *ostg, *bbuf, *pbuf;
+    const uint8_t *tabs;  // NVFP4 decoding tables
     int *linfo, *oinfo, *tinfo;
     uint32_t tmem;
 
-    __device__ Pass2(const KGeom &g_, const PipeSmem &ps_, int *wd_, uint32_t tmem_base) : g(g_), ps(ps_), wd(wd_) {
+    __device__ Pass2(const KGeom &g_, const PipeSmem &ps_, int *wd_, uint32_t tmem_base, const uint8_t *tabs_)
+        : g(g_), ps(ps_), wd(wd_), tabs(tabs_) {
         land = ps.base;
-        opnd = land + NL * TB;
+        opnd = land + NLS * C::LSLOT;
         ostg = opnd + NO * 2 * TB;
         bbuf = ostg + TB;
         pbuf = bbuf + 2 * C::IMG;
@@ -673,7 +802,7 @@ struct Pass2 {
         tinfo = oinfo + 6 * NO;
         tmem = tmem_base;
     }
-    __device__ uint8_t *lq(int s) const { return land + s * SPAN * TB; }
+    __device__ uint8_t *lq(int s) const { return land + s * C::LSLOT; }
     __device__ uint8_t *oq(int s) const { return opnd + s * 2 * TB; }
     __device__ uint8_t *oph(int s) const { return opnd + s * 2 * TB + TB; }
     __device__ uint32_t bar(int i) const { return ptx::smem_u32(ps.bars + i); }
@@ -767,6 +896,8 @@ struct Pass2 {
                     ptx::mbar_arrive(tfull(ti));
                 }
                 if (!ok) break;
+                ScaleSpan sp{};  // NVFP4: the span's scale bytes, rounded outwards to 16 B
+                if constexpr (FP4) sp = scale_span<D>((long long)bh * g.N + n, SPAN * kTile, (long long)g.BH * g.N);
                 int *inf = linfo + 8 * sl;  // for the transform warps
                 inf[0] = u;
                 inf[1] = t0;
@@ -774,9 +905,11 @@ struct Pass2 {
                 inf[3] = nu;
                 inf[4] = n;
                 inf[5] = L - (t_lo + t0) * kTile;  // rows of the span inside the block (may exceed the span)
+                inf[6] = sp.off;
                 const MapCoord mc = map_coord(n, hh, g.swap_q);
-                ptx::mbar_arrive_expect_tx(lfull(sl), SPAN * TB);
+                ptx::mbar_arrive_expect_tx(lfull(sl), FP4 ? F::DB + sp.bytes : SPAN * TB);
                 ptx::tma_load_4d_hint(ptx::smem_u32(lq(sl)), mq, lfull(sl), 0, mc.y, mc.z, bb, policy);
+                if constexpr (FP4) ptx::bulk_load(ptx::smem_u32(lq(sl) + F::DB), g.sq_scale + sp.a0, sp.bytes, lfull(sl));
                 if (p == early - 1 && !(ok = issue_prefix(bh, b))) break;
             }
             ++nu;
@@ -888,7 +1021,11 @@ struct Pass2 {
                 }
                 uint32_t w[D / 2], ph[D / 2];
                 const bool live = r < valid;
-                if (live) load_row<D>(lq(sl) + h * TB, r, w);
+                if constexpr (FP4) {
+                    if (live) fp4_row<D>(lq(sl) + r * (D / 2), lq(sl) + F::DB + ld_volatile(inf + 6) + r * F::S1, tabs, w);
+                } else {
+                    if (live) load_row<D>(lq(sl) + h * TB, r, w);
+                }
                 if (h == hmax - 1) {
                     // the next TMA into this slot writes through the async proxy: order this
                     // thread's generic reads of the slot before it
@@ -954,12 +1091,18 @@ struct Pass2 {
             const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
             float zh, zl;
             tmem_ld_2cols(taddr + D, zh, zl);
-            const float inv = __frcp_rn(zh + zl + g.eps);
+            // NVFP4: phi(q) carries the global scale gq (numerator and denominator alike)
+            const float gq = FP4 ? g.gq : 1.0f;
+            const float inv = FP4 ? __frcp_rn(gq * zh + gq * zl + g.eps) : __frcp_rn(zh + zl + g.eps);
             uint32_t ow[D / 2];
 #pragma unroll
             for (int half = 0; half < D / 32; ++half) {
                 float v[32];
                 ptx::tmem_ld_32cols(taddr + 32 * half, v);
+                if constexpr (FP4) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q] *= gq;
+                }
 #pragma unroll
                 for (int q = 0; q < 16; ++q) ow[16 * half + q] = pack_bf16x2(v[2 * q] * inv, v[2 * q + 1] * inv);
             }
@@ -995,7 +1138,7 @@ struct Cta {
         ctrl = base + off_ctrl;
         flags = reinterpret_cast<volatile int *>(ctrl + Cfg::OFF_FLAGS);
         tmem_slot = reinterpret_cast<uint32_t *>(ctrl + Cfg::OFF_FLAGS + 4);
-        s_tab = reinterpret_cast<float2 *>(ctrl + Cfg::CTRL);
+        s_tab = reinterpret_cast<float2 *>(ctrl + Cfg::CTRL + Cfg::TABS);
     }
     __device__ PipeSmem pipe(int p, int pipe_bytes, uint8_t *ones) const {
         PipeSmem ps;
@@ -1009,12 +1152,12 @@ struct Cta {
 };
 
 // Pass 1: chunk partial states.  Persistent, one CTA per SM, NP pipelines.
-template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(K1Cfg<D>::THREADS, 1)
+template <int D, int PT, int PY, int PX, bool FP4>
+__global__ void __launch_bounds__(K1Cfg<D, FP4>::THREADS, 1)
     partial_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                       const __grid_constant__ KGeom g, int *watchdog) {
-    using C = K1Cfg<D>;
-    using P = Pass1<D, PT, PY, PX>;
+    using C = K1Cfg<D, FP4>;
+    using P = Pass1<D, PT, PY, PX, FP4>;
     extern __shared__ uint8_t smem_raw[];
     Cta<C> cta(smem_raw, C::OFF_CTRL);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1036,20 +1179,22 @@ __global__ void __launch_bounds__(K1Cfg<D>::THREADS, 1)
     if (tid == 0) griddep_launch_dependents();
     const PipeSmem ps = cta.pipe(pipe, C::PIPE, ones);
     const uint32_t tmem = tmem_base + pipe * C::NA * C::ACOLS;
+    uint8_t *tabs = cta.ctrl + C::CTRL;  // NVFP4 decoding tables
     if (pw < 4) {
         const int r = tid & 127, ntrans = 128 * C::NP, tt = pipe * 128 + r;
         const RopeTab tab = load_rope_tab<PT, PY, PX>(g, cta.s_tab, tt, ntrans);
+        if constexpr (FP4) fill_fp4_tables(tabs, tt, ntrans);
         uint4 *o4 = reinterpret_cast<uint4 *>(ones);  // all 1.0, so its swizzle is irrelevant
         for (int i = tt; i < C::TB / 16; i += ntrans) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
         ptx::fence_proxy_async_smem();  // the ones block is read by the MMA (async proxy)
         ptx::named_bar_sync(kBarTab, ntrans);
-        P(g, ps, watchdog, tmem).transform(tab, r);
+        P(g, ps, watchdog, tmem, tabs).transform(tab, r);
     } else if (pw < 8) {
-        P(g, ps, watchdog, tmem).epilogue(tid & 127, warp & 3);
+        P(g, ps, watchdog, tmem, tabs).epilogue(tid & 127, warp & 3);
     } else if (pw == 8) {
-        if (lane < 2) P(g, ps, watchdog, tmem).producer(&mk, &mv, lane);
+        if (lane < 2) P(g, ps, watchdog, tmem, tabs).producer(&mk, &mv, lane);
     } else if (lane == 0) {
-        P(g, ps, watchdog, tmem).mma();
+        P(g, ps, watchdog, tmem, tabs).mma();
     }
     ptx::tc_fence_before_sync();
     __syncthreads();
@@ -1062,12 +1207,12 @@ __global__ void __launch_bounds__(K1Cfg<D>::THREADS, 1)
 // Pass 2: outputs.  Persistent, one CTA per SM, NP pipelines; launched with
 // programmatic dependent launch, it reads the prefix states only after
 // griddepcontrol.wait (the block scan before it has finished).
-template <int D, int PT, int PY, int PX>
-__global__ void __launch_bounds__(K2Cfg<D>::THREADS, 1)
+template <int D, int PT, int PY, int PX, bool FP4>
+__global__ void __launch_bounds__(K2Cfg<D, FP4>::THREADS, 1)
     output_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ KGeom g, __nv_bfloat16 *o,
                      int *watchdog) {
-    using C = K2Cfg<D>;
-    using P = Pass2<D, PT, PY, PX>;
+    using C = K2Cfg<D, FP4>;
+    using P = Pass2<D, PT, PY, PX, FP4>;
     extern __shared__ uint8_t smem_raw[];
     Cta<C> cta(smem_raw, C::OFF_CTRL);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1087,19 +1232,21 @@ __global__ void __launch_bounds__(K2Cfg<D>::THREADS, 1)
     const uint32_t tmem_base = *cta.tmem_slot;
     const PipeSmem ps = cta.pipe(pipe, C::PIPE, nullptr);
     const uint32_t tmem = tmem_base + pipe * C::NA * C::ACOLS;
+    uint8_t *tabs = cta.ctrl + C::CTRL;  // NVFP4 decoding tables
     if (pw < 4) {
         const int r = tid & 127, ntrans = 128 * C::NP;
         const RopeTab tab = load_rope_tab<PT, PY, PX>(g, cta.s_tab, pipe * 128 + r, ntrans);
+        if constexpr (FP4) fill_fp4_tables(tabs, pipe * 128 + r, ntrans);
         ptx::named_bar_sync(kBarTab, ntrans);
-        P(g, ps, watchdog, tmem).transform(tab, r);
+        P(g, ps, watchdog, tmem, tabs).transform(tab, r);
     } else if (pw < 8) {
         // pass 1 and the scan, which this kernel may overlap, touch neither Q nor O: only
         // the prefix read (in the producer) waits for them
-        P(g, ps, watchdog, tmem).epilogue(o, warp & 3, lane);
+        P(g, ps, watchdog, tmem, tabs).epilogue(o, warp & 3, lane);
     } else if (pw == 8) {
-        if (lane == 0) P(g, ps, watchdog, tmem).producer(&mq);
+        if (lane == 0) P(g, ps, watchdog, tmem, tabs).producer(&mq);
     } else if (lane == 0) {
-        P(g, ps, watchdog, tmem).mma();
+        P(g, ps, watchdog, tmem, tabs).mma();
     }
     ptx::tc_fence_before_sync();
     __syncthreads();

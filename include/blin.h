@@ -207,6 +207,41 @@ BLIN_API blin_status blin_block_step_strided(const void *q, const void *k, const
                                              const blin_layout *o_layout, blin_state *st, int commit,
                                              blin_stream stream);
 
+/* ---------------------------------------------------------------- NVFP4 inputs */
+
+/* One NVFP4 operand [B][H][N][d] (news article, NVFP4 / SVDQuant paragraph: the
+ * QKV projections run in NVFP4).  Element i of a token's d-vector is
+ *   e2m1(code_i) * e4m3(scale[i / 16]) * global_scale
+ * with code_i the E2M1 nibble i of the token's d/2 data bytes (even elements
+ * in the low nibble; bit 3 sign, bits 2..1 exponent, bit 0 mantissa) and
+ * scale the token's d/16 E4M3 bytes (one per 16 consecutive elements).
+ *   data   device [B][H][N][d/2] bytes, 16-byte aligned
+ *   scale  device [B][H][N][d/16] bytes, 16-byte aligned; the allocation must
+ *          be a whole number of 16-byte units (scale bytes are copied in
+ *          aligned 16-byte runs)
+ *   global_scale  finite, > 0 */
+typedef struct {
+    const void *data;
+    const void *scale;
+    float global_scale;
+} blin_nvfp4;
+
+/* blin_prefill on NVFP4 q, k, v; o is bf16 [B][H][N][d].  The tensor-core
+ * kernels decode the 4-bit values in shared memory (E2M1 x E4M3 products are
+ * exact in bf16) and apply the global scales in fp32, so a token-head moves
+ * 3 * (d/2 + d/16) + 2d bytes instead of 8d.  Needs the tensor-core path (the
+ * compiled RoPE splits), else BLIN_ERR_SHAPE.  Workspace and state as for
+ * blin_prefill; with power-of-two global scales the results are bitwise those
+ * of blin_prefill on the decoded bf16 values. */
+BLIN_API blin_status blin_prefill_nvfp4(const blin_nvfp4 *q, const blin_nvfp4 *k, const blin_nvfp4 *v, void *o,
+                                        int B, int H, int d, const blin_geom *g, blin_state *st, void *workspace,
+                                        size_t ws_bytes, blin_stream stream);
+
+/* blin_block_step on NVFP4 q, k, v (see blin_prefill_nvfp4); o is bf16. */
+BLIN_API blin_status blin_block_step_nvfp4(const blin_nvfp4 *q, const blin_nvfp4 *k, const blin_nvfp4 *v, void *o,
+                                           int B, int H, int d, const blin_geom *g, blin_state *st, int commit,
+                                           blin_stream stream);
+
 /* ---------------------------------------------------------------- causal temporal convolution */
 
 /* The Mix-FFN's causal block temporal convolution and its one-frame cache

@@ -22,7 +22,7 @@ FAKE = 1 << 20  # a 16-byte aligned non-NULL address that is never dereferenced
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(blin_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(blin_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
