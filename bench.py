@@ -19,7 +19,9 @@ oracle's CPU rate and the SM clocks seen while timing, plus sub-records:
   denoise      16 blocks, each denoised by 4 read-only block steps (fresh
                Q/K/V, commit=0) and then committed once, replayed as a graph;
   tconv        the Mix-FFN's causal block temporal convolution over the same
-               latent video (C = 2240 channels), bytes against the HBM peak.
+               latent video (C = 2240 channels), bytes against the HBM peak;
+  nvfp4_720p   the 720p prefill on NVFP4 Q/K/V (4-bit codes with block
+               scales): 118 instead of 256 bytes per token-head.
 
 With N > 1 GPUs every rank runs its own independent copy of the workload (weak
 scaling; heads and videos never exchange data) and each time is the max over
@@ -643,6 +645,54 @@ def measure_tconv(args, w, torch, blin, world, rank, clk):
                          "algorithmic_bytes_per_launch": alg}}
 
 
+def measure_nvfp4(args, w, torch, blin, world, rank, clk):
+    """The prefill on NVFP4 Q/K/V (packed E2M1 codes, one E4M3 scale per 16 elements, a global
+    scale per tensor; bf16 output): time per step and algorithmic bytes against the HBM peak."""
+    wr = replica_workload(w, rank)
+    ops = [blin.Nvfp4Tensor(torch.from_numpy(dt), torch.from_numpy(sc), gs)
+           for dt, sc, gs in workloads.nvfp4_call_tensors(wr)]
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device="cuda")
+    grid = (w.T, w.Hg, w.Wg)
+    ws = torch.empty(blin.workspace_size(w.B, w.H, w.d, grid, w.F, w.split, w.theta, w.eps), dtype=torch.uint8,
+                     device="cuda")
+    geom = blin._geom(w.T, w.Hg, w.Wg, w.F, w.split, w.theta, w.eps)
+    cs = [o.c() for o in ops]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    cargs = (ctypes.byref(cs[0]), ctypes.byref(cs[1]), ctypes.byref(cs[2]), ctypes.c_void_p(out.data_ptr()), w.B,
+             w.H, w.d, ctypes.byref(geom), None, ctypes.c_void_p(ws.data_ptr()), ws.numel(), stream)
+    call = blin.lib.blin_prefill_nvfp4
+
+    def step():
+        rc = call(*cargs)
+        if rc != 0:
+            raise RuntimeError(blin.lib.blin_last_error().decode())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall = time.time()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clk.timed(t_wall, time.time())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    units = w.B * w.H * w.N
+    per_unit = 3 * (w.d // 2 + w.d // 16) + 2 * w.d  # q, k, v packed codes and scales read; bf16 o written
+    alg = units * per_unit
+    peak, peak_kind = hbm_peak()
+    return {"workload": f"{w.name} prefill with NVFP4 q, k, v (E2M1 + E4M3 per 16 elements + global scale), "
+                        f"bf16 o: B={w.B} H={w.H} d={w.d}, latent {w.T}x{w.Hg}x{w.Wg}, blocks of {w.F} frames",
+            "ms_per_step": ms, "value": job_throughput(units, world, ms), "unit": UNIT,
+            "bytes_per_token_head": per_unit,
+            "roofline": {"bound": "hbm", "kernel": "whole step (3 launches)", "achieved": alg / (ms * 1e-3) / 1e9,
+                         "peak": peak, "unit": "GB/s", "frac": alg / (ms * 1e-3) / 1e9 / peak,
+                         "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_step": alg}}
+
+
 def run_blin(args):
     torch, blin, world, rank, local = _load_blin(args)
     main_name = "720p" if args.config == "all" else args.config
@@ -672,6 +722,7 @@ def run_blin(args):
             subs["denoise"] = measure_decode(args, workloads.CONFIGS["decode"].with_(steps=16), torch, blin, world,
                                              rank, clk, 4)
             subs["tconv"] = measure_tconv(args, workloads.CONV_CONFIGS["conv-480p"], torch, blin, world, rank, clk)
+            subs["nvfp4_720p"] = measure_nvfp4(args, workloads.CONFIGS["720p"], torch, blin, world, rank, clk)
         time.sleep(0.25)
     line = {"metric": main.pop("metric"), "value": main.pop("value"), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main.pop("ms_per_step"),

@@ -93,10 +93,11 @@ static int tc_chunks(long long L, int d) {
     const long long ct = d == 32 ? kChunkTiles32 : kChunkTiles64;
     return (int)std::max(1LL, (nt + ct - 1) / ct);
 }
-// Tensor-core path, pass 2: query groups of up to kGroupTiles tiles per block.
-static int tc_groups(long long L) {
+// Tensor-core path, pass 2: query groups of up to `gt` tiles per block (the
+// grouping does not change any output bit).
+static int tc_groups(long long L, int gt) {
     const long long nt = (L + kTile - 1) / kTile;
-    return (int)std::max(1LL, (nt + kGroupTiles - 1) / kGroupTiles);
+    return (int)std::max(1LL, (nt + gt - 1) / gt);
 }
 // CUDA-core path: 1024-token chunks.
 static int simt_chunks(long long L) { return (int)std::max(1LL, (L + kChunk - 1) / kChunk); }
@@ -153,9 +154,16 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
         g.nc_first = chunks(Lf);
         g.nc_mid = chunks(Lm);
         g.nc_last = chunks(Ll);
-        g.ng_first = tc_groups(Lf);
-        g.ng_mid = tc_groups(Lm);
-        g.ng_last = tc_groups(Ll);
+        // query groups of 8 tiles (the B operand is rebuilt once per group), fewer when
+        // the call has too few groups to keep every pass-2 pipeline of a B200 busy
+        int gt = 8;
+        auto all_groups = [&](int t) {
+            return (long long)g.BH * (tc_groups(Lf, t) + (long long)mids * tc_groups(Lm, t) + (g.nblk >= 2 ? tc_groups(Ll, t) : 0));
+        };
+        while (gt > 2 && all_groups(gt) < 3 * 296) gt /= 2;
+        g.ng_first = tc_groups(Lf, gt);
+        g.ng_mid = tc_groups(Lm, gt);
+        g.ng_last = tc_groups(Ll, gt);
         g.U1 = g.nblk == 0 ? 0 : g.nc_first + mids * g.nc_mid + (g.nblk >= 2 ? g.nc_last : 0);
         g.U2 = g.nblk == 0 ? 0 : g.ng_first + mids * g.ng_mid + (g.nblk >= 2 ? g.ng_last : 0);
         g.cpb = std::max(g.nc_first, g.nblk >= 2 ? g.nc_last : 0);
@@ -323,8 +331,7 @@ static blin_status run(Plan &p, const void *q, const void *k, const void *v, voi
             maps = make_map4_fp4(&mq, q, B, g.H, g.N, d, kTile) && make_map4_fp4(&mk, k, B, g.H, g.N, d, kTile) &&
                    make_map4_fp4(&mv, v, B, g.H, g.N, d, kTile);
         } else {
-            // pass 2 lands Q in spans of tiles (one box each: 256 rows at d = 32, 128 at d = 64)
-            maps = make_map4(&mq, q, g.lq, B, g.H, g.N, d, d == 32 ? 2 * kTile : kTile, &g.swap_q) &&
+            maps = make_map4(&mq, q, g.lq, B, g.H, g.N, d, kTile, &g.swap_q) &&
                    make_map4(&mk, k, g.lq, B, g.H, g.N, d, kTile, &sk) && make_map4(&mv, v, g.lq, B, g.H, g.N, d, kTile, &sv);
         }
         if (!maps)

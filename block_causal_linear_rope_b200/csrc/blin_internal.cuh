@@ -16,8 +16,6 @@ constexpr int kTile = 128;
 // CUDA-core path: state chunks of 1024 tokens counted from the start of their
 // block (a function of the block alone, so streamed calls reduce like prefill).
 constexpr int kChunk = 1024;
-// Tensor-core path: query tiles per output group.
-constexpr int kGroupTiles = 4;
 
 // Element strides of one [B][H][N][d] operand (d innermost, stride 1).
 struct Layout {

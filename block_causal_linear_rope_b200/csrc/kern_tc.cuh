@@ -66,14 +66,15 @@ struct TokPos {
     }
 };
 
-// A CTA's shared-memory RoPE table: (cos, sin) of every (position, pair) of
-// the call's frame window and of every row and column, one section per axis.
-// Each section is stored pair-major ([pair][position]) so that the threads of
-// a warp, which hold consecutive tokens and hence mostly consecutive columns,
-// read consecutive words: no bank conflicts on the x section, broadcasts on t, y.
+// A CTA's shared-memory RoPE table: (cos, sin) of every (position, pair) of the
+// call's frame window and of every row and column, one section per axis, each
+// position-major ([position][pair], the order rope_entry enumerates).  A token row
+// reads its position's pairs two at a time (16-byte loads at an offset known at
+// compile time from one base per axis); across a warp the t and y entries are
+// mostly broadcasts, and consecutive columns sit 48 bytes apart (d = 32), which
+// the 16-byte loads of a quarter-warp take without bank conflicts.
 struct RopeTab {
-    const float2 *t, *y, *x;  // t indexed by relative frame (window offset folded in)
-    int nt, ny, nx;            // positions per pair in each section (T, Hg, Wg)
+    const float4 *t, *y, *x;  // section bases; t indexed by relative frame (window offset folded in)
 };
 
 // Fills this CTA's shared-memory RoPE table (the tensor-core path is only
@@ -81,27 +82,13 @@ struct RopeTab {
 // follow).  Entry values are those of rope_entry (same order of operations).
 template <int PT, int PY, int PX>
 __device__ __forceinline__ RopeTab load_rope_tab(const KGeom &g, float2 *s_tab, int tid, int nthreads) {
-    const int nt = g.T * PT, ny = g.Hg * PY, n = nt + ny + g.Wg * PX;
-    for (int i = tid; i < n; i += nthreads) {
-        int src;  // index of the same entry in the position-major order rope_entry enumerates
-        if (i < nt) {
-            src = (i % g.T) * PT + i / g.T;
-        } else if (i < nt + ny) {
-            const int r = i - nt;
-            src = nt + (r % g.Hg) * PY + r / g.Hg;
-        } else {
-            const int r = i - nt - ny;
-            src = nt + ny + (r % g.Wg) * PX + r / g.Wg;
-        }
-        s_tab[i] = rope_entry(src, g.T, g.t0, g.Hg, PT, PY, PX, g.theta);
-    }
+    static_assert(PT % 2 == 0 && PY % 2 == 0 && PX % 2 == 0, "pairs are read two at a time");
+    const int n = g.T * PT + g.Hg * PY + g.Wg * PX;
+    for (int i = tid; i < n; i += nthreads) s_tab[i] = rope_entry(i, g.T, g.t0, g.Hg, PT, PY, PX, g.theta);
     RopeTab r;
-    r.t = s_tab;
-    r.y = s_tab + g.tab_y;
-    r.x = s_tab + g.tab_x;
-    r.nt = g.T;
-    r.ny = g.Hg;
-    r.nx = g.Wg;
+    r.t = reinterpret_cast<const float4 *>(s_tab);
+    r.y = reinterpret_cast<const float4 *>(s_tab + g.tab_y);
+    r.x = reinterpret_cast<const float4 *>(s_tab + g.tab_x);
     return r;
 }
 
@@ -114,24 +101,30 @@ template <int D, int PT, int PY, int PX, bool ZP>
 __device__ __forceinline__ void phi_rope_row(uint32_t (&w)[D / 2], uint32_t (&ph)[D / 2], const RopeTab &tab,
                                              const TokPos &tp, float *zp) {
     static_assert(PT + PY + PX == D / 2, "split must cover d");
-    const float2 *rt = tab.t + tp.t;
-    const float2 *ry = tab.y + tp.y;
-    const float2 *rx = tab.x + tp.x;
+    const float4 *rt = tab.t + tp.t * (PT / 2);
+    const float4 *ry = tab.y + tp.y * (PY / 2);
+    const float4 *rx = tab.x + tp.x * (PX / 2);
 #pragma unroll
-    for (int p = 0; p < D / 2; ++p) {
-        const float2 cs = p < PT ? rt[p * tab.nt] : (p < PT + PY ? ry[(p - PT) * tab.ny] : rx[(p - PT - PY) * tab.nx]);
-        // ReLU on the packed pair (exact), then widen
-        __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162 *>(&w[p]);
-        hv = __hmax2(hv, __float2bfloat162_rn(0.f));
-        const uint32_t u = *reinterpret_cast<uint32_t *>(&hv);
-        ph[p] = u;
-        const float a = __uint_as_float(u << 16);
-        const float b = __uint_as_float(u & 0xFFFF0000u);
-        if constexpr (ZP) {
-            zp[2 * p] += a;
-            zp[2 * p + 1] += b;
+    for (int q = 0; q < D / 4; ++q) {  // pairs 2q, 2q + 1 (never straddling two axes)
+        const int p0 = 2 * q;
+        const float4 cs2 = p0 < PT ? rt[q] : (p0 < PT + PY ? ry[q - PT / 2] : rx[q - (PT + PY) / 2]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int p = p0 + h;
+            const float c = h ? cs2.z : cs2.x, sn = h ? cs2.w : cs2.y;
+            // ReLU on the packed pair (exact), then widen
+            __nv_bfloat162 hv = *reinterpret_cast<__nv_bfloat162 *>(&w[p]);
+            hv = __hmax2(hv, __float2bfloat162_rn(0.f));
+            const uint32_t u = *reinterpret_cast<uint32_t *>(&hv);
+            ph[p] = u;
+            const float a = __uint_as_float(u << 16);
+            const float b = __uint_as_float(u & 0xFFFF0000u);
+            if constexpr (ZP) {
+                zp[2 * p] += a;
+                zp[2 * p + 1] += b;
+            }
+            w[p] = pack_bf16x2(fmaf(a, c, -b * sn), fmaf(a, sn, b * c));
         }
-        w[p] = pack_bf16x2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
     }
 }
 
@@ -283,7 +276,7 @@ struct TcCfg {
     static constexpr uint32_t TCOLS = 512;
     static constexpr int E = D * D + D, E4 = E / 4;
     // control block: [NP][BARS_PER_PIPE] mbarriers, 16 B of flags, [NP][INFO_PER_PIPE] record ints
-    static constexpr int BARS_PER_PIPE = 64;
+    static constexpr int BARS_PER_PIPE = 72;
     static constexpr int INFO_PER_PIPE = 160;
     static constexpr int OFF_FLAGS = NP * BARS_PER_PIPE * 8;
     static constexpr int OFF_INFO = OFF_FLAGS + 16;
@@ -332,10 +325,9 @@ template <int D, bool FP4 = false>
 struct K2Cfg : TcCfg<D> {
     using B = TcCfg<D>;
     using F = Fp4Tile<D>;
-    // bf16 Q lands in slots of SPAN consecutive tiles, one TMA box each (fewer, larger
-    // boxes); NVFP4 Q in slots of one tile's data and scales
-    static constexpr int SPAN = FP4 ? 1 : (D == 32 ? 2 : 1);  // tiles per Q landing slot
-    static constexpr int NLS = FP4 ? 8 : 3;                    // Q landing slots
+    // Q lands one tile per slot (bf16: one TMA box; NVFP4: a tile's data and scales)
+    static constexpr int SPAN = 1;                             // tiles per Q landing slot
+    static constexpr int NLS = FP4 ? 8 : (D == 32 ? 5 : 3);    // Q landing slots
     static constexpr int LSLOT = FP4 ? (F::DB + F::SB + 1023) / 1024 * 1024 : SPAN * B::TB;
     static constexpr int NL = NLS * SPAN;                      // Q tiles in the landing ring
     static constexpr int NT = B::NA > B::NO + 1 ? B::NA : B::NO + 1;  // tile-done barriers
@@ -343,12 +335,13 @@ struct K2Cfg : TcCfg<D> {
     static constexpr int BATOM = OutB<D>::BATOM;
     static constexpr int IMG = OutB<D>::IMG;
     static constexpr int PRE = (D * D + D) * 4;            // one fp32 prefix state (S, z)
-    // Q ring, operand ring, O staging (4 warps x 32 rows), 2 B images, prefix state
-    static constexpr int PIPE = (NLS * LSLOT + B::NO * 2 * B::TB + B::TB + 2 * IMG + PRE + 1023) / 1024 * 1024;
+    // Q ring, operand ring, O staging (4 warps x 32 rows), 2 B images, 2 prefix states
+    // (a group's prefix is fetched while the previous group is still being computed)
+    static constexpr int PIPE = (NLS * LSLOT + B::NO * 2 * B::TB + B::TB + 2 * IMG + 2 * PRE + 1023) / 1024 * 1024;
     static constexpr int OFF_CTRL = B::NP * PIPE;
     static constexpr int TABS = FP4 ? F::TABS : 0;
     static constexpr int FIXED = OFF_CTRL + B::CTRL + TABS + 1024;
-    static constexpr int NBAR = 2 * NLS + B::NO + NT + B::NA + 4 + 2 * B::NINFO + 1;
+    static constexpr int NBAR = 2 * NLS + B::NO + NT + B::NA + 6 + 2 * B::NINFO + 1;
     static constexpr int NINF = 8 * NLS + 6 * B::NO + 4 * B::NINFO;
     static_assert(NBAR <= B::BARS_PER_PIPE && NINF <= B::INFO_PER_PIPE, "control block");
 };
@@ -811,12 +804,14 @@ struct Pass2 {
     __device__ uint32_t ofull(int s) const { return bar(2 * NLS + s); }
     __device__ uint32_t tdone(int s) const { return bar(2 * NLS + NO + s); }
     __device__ uint32_t acce(int a) const { return bar(2 * NLS + NO + NT + a); }
-    __device__ uint32_t pfull() const { return bar(2 * NLS + NO + NT + NA); }
-    __device__ uint32_t pempty() const { return bar(2 * NLS + NO + NT + NA + 1); }
-    __device__ uint32_t bempty(int s) const { return bar(2 * NLS + NO + NT + NA + 2 + s); }
-    __device__ uint32_t tfull(int i) const { return bar(2 * NLS + NO + NT + NA + 4 + i); }
-    __device__ uint32_t tempty(int i) const { return bar(2 * NLS + NO + NT + NA + 4 + C::NINFO + i); }
-    __device__ uint32_t drain() const { return bar(2 * NLS + NO + NT + NA + 4 + 2 * C::NINFO); }
+    // pfull[s] / pempty[s]: prefix buffer s landed / turned into a B image (4 warps)
+    __device__ uint32_t pfull(int s) const { return bar(2 * NLS + NO + NT + NA + s); }
+    __device__ uint32_t pempty(int s) const { return bar(2 * NLS + NO + NT + NA + 2 + s); }
+    __device__ uint32_t bempty(int s) const { return bar(2 * NLS + NO + NT + NA + 4 + s); }
+    __device__ uint32_t tfull(int i) const { return bar(2 * NLS + NO + NT + NA + 6 + i); }
+    __device__ uint32_t tempty(int i) const { return bar(2 * NLS + NO + NT + NA + 6 + C::NINFO + i); }
+    __device__ uint32_t drain() const { return bar(2 * NLS + NO + NT + NA + 6 + 2 * C::NINFO); }
+    __device__ uint8_t *prefix_buf(int s) const { return pbuf + s * C::PRE; }
 
     __device__ static void init_barriers(uint64_t *b) {
         auto at = [&](int i) { return ptx::smem_u32(b + i); };
@@ -827,14 +822,16 @@ struct Pass2 {
         for (int s = 0; s < NO; ++s) ptx::mbar_init(at(2 * NLS + s), 4);           // ofull
         for (int s = 0; s < NT; ++s) ptx::mbar_init(at(2 * NLS + NO + s), 1);      // tdone: commit
         for (int a = 0; a < NA; ++a) ptx::mbar_init(at(2 * NLS + NO + NT + a), 4);  // acce: epilogue
-        ptx::mbar_init(at(2 * NLS + NO + NT + NA), 1);                              // pfull: bulk copy
-        ptx::mbar_init(at(2 * NLS + NO + NT + NA + 1), 4);                          // pempty: transform
-        for (int s = 0; s < 2; ++s) ptx::mbar_init(at(2 * NLS + NO + NT + NA + 2 + s), 1);  // bempty: commit
-        for (int i = 0; i < C::NINFO; ++i) {
-            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + i), 1);              // tfull: producer
-            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + C::NINFO + i), 4);  // tempty: epilogue
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + s), 1);      // pfull: bulk copy
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 2 + s), 4);  // pempty: transform
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + s), 1);  // bempty: commit
         }
-        ptx::mbar_init(at(2 * NLS + NO + NT + NA + 4 + 2 * C::NINFO), 1);  // drain
+        for (int i = 0; i < C::NINFO; ++i) {
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 6 + i), 1);              // tfull: producer
+            ptx::mbar_init(at(2 * NLS + NO + NT + NA + 6 + C::NINFO + i), 4);  // tempty: epilogue
+        }
+        ptx::mbar_init(at(2 * NLS + NO + NT + NA + 6 + 2 * C::NINFO), 1);  // drain
     }
 
     __device__ int ng_of(int b) const { return units_of_block(g, b, g.ng_first, g.ng_mid, g.ng_last); }
@@ -848,15 +845,18 @@ struct Pass2 {
         const int total = g.BH * g.U2;
         int kp = 0, j = 0, nu = 0, npre = 0;
         bool ok = true, waited = false;
-        // the group's fp32 prefix state (written by the block scan, the previous kernel)
+        // group nu's fp32 prefix state (written by the block scan, the previous kernel) into
+        // buffer nu & 1, as soon as group nu - 2 has turned that buffer into its B image
         auto issue_prefix = [&](int bh, int b) {
-            if (nu >= 1 && !ptx::mbar_wait_bounded(pempty(), (nu - 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs)) return false;
+            const int ps_ = nu & 1;
+            if (nu >= 2 && !ptx::mbar_wait_bounded(pempty(ps_), ((nu >> 1) - 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs))
+                return false;
             if (!waited) {
                 griddep_wait();
                 waited = true;
             }
-            ptx::mbar_arrive_expect_tx(pfull(), C::PRE);
-            ptx::bulk_load(ptx::smem_u32(pbuf), g.prefix + ((size_t)bh * g.nblk + b) * E, C::PRE, pfull());
+            ptx::mbar_arrive_expect_tx(pfull(ps_), C::PRE);
+            ptx::bulk_load(ptx::smem_u32(prefix_buf(ps_)), g.prefix + ((size_t)bh * g.nblk + b) * E, C::PRE, pfull(ps_));
             ++npre;
             return true;
         };
@@ -872,8 +872,8 @@ struct Pass2 {
             const int t_lo = gi * nt / ng, t_hi = (gi + 1) * nt / ng, ntiles = t_hi - t_lo;
             const int nspans = (ntiles + SPAN - 1) / SPAN;
             const int bb = bh / g.H, hh = bh - bb * g.H;
-            // Q spans do not depend on the prefix: the first few go out before it
-            const int early = min(nspans, NLS);
+            // the prefix first: it is needed before the group's first tile can be multiplied
+            if (!(ok = issue_prefix(bh, b))) break;
             for (int p = 0; p < nspans; ++p, ++kp) {
                 const int sl = kp % NLS;
                 if (kp >= NLS && !ptx::mbar_wait_bounded(lempty(sl), ((kp / NLS) - 1) & 1, wd, WD_P2_EMPTY, kWaitLimitNs)) {
@@ -910,7 +910,6 @@ struct Pass2 {
                 ptx::mbar_arrive_expect_tx(lfull(sl), FP4 ? F::DB + sp.bytes : SPAN * TB);
                 ptx::tma_load_4d_hint(ptx::smem_u32(lq(sl)), mq, lfull(sl), 0, mc.y, mc.z, bb, policy);
                 if constexpr (FP4) ptx::bulk_load(ptx::smem_u32(lq(sl) + F::DB), g.sq_scale + sp.a0, sp.bytes, lfull(sl));
-                if (p == early - 1 && !(ok = issue_prefix(bh, b))) break;
             }
             ++nu;
         }
@@ -933,7 +932,8 @@ struct Pass2 {
         const int oldest = marked ? kp - NLS + 1 : kp - NLS;
         for (int kk = kp - 1; kk >= 0 && kk >= oldest; --kk)
             ptx::mbar_wait_bounded(lfull(kk % NLS), (kk / NLS) & 1, wd, WD_P2_FULL, kWaitLimitNs);
-        if (npre > 0) ptx::mbar_wait_bounded(pfull(), (npre - 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs);
+        for (int j2 = npre - 1; j2 >= 0 && j2 >= npre - 2; --j2)
+            ptx::mbar_wait_bounded(pfull(j2 & 1), (j2 >> 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs);
     }
 
     // ------------------------------------------------------------ MMA issuer (one thread)
@@ -1008,16 +1008,16 @@ struct Pass2 {
                     const int bs = ord & 1;
                     if ((ord >= 2 && !ptx::mbar_wait_bounded(bempty(bs), ((ord >> 1) - 1) & 1, wd, WD_P2_BREADY,
                                                              kWaitLimitNs)) ||
-                        !ptx::mbar_wait_bounded(pfull(), ord & 1, wd, WD_P2_BREADY, kWaitLimitNs)) {
+                        !ptx::mbar_wait_bounded(pfull(ord & 1), (ord >> 1) & 1, wd, WD_P2_BREADY, kWaitLimitNs)) {
                         abort = true;
                         break;
                     }
-                    const float *pre = reinterpret_cast<const float *>(pbuf);
+                    const float *pre = reinterpret_cast<const float *>(prefix_buf(ord & 1));
                     uint4 *dst = reinterpret_cast<uint4 *>(bbuf + bs * C::IMG);
                     for (int item = r; item < C::IMG / 16; item += 128) dst[item] = b_operand_chunk<D>(pre, item);
                     // the next bulk copy into the prefix buffer writes through the async proxy
                     ptx::fence_proxy_async_smem();  // also: the B image is read by the MMA (ordered by ofull)
-                    warp_arrive(pempty(), lane);
+                    warp_arrive(pempty(ord & 1), lane);
                 }
                 uint32_t w[D / 2], ph[D / 2];
                 const bool live = r < valid;
@@ -1089,16 +1089,16 @@ struct Pass2 {
             }
             ptx::tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * sub) << 16) + a * C::ACOLS;
-            float zh, zl;
-            tmem_ld_2cols(taddr + D, zh, zl);
+            // the denominator's two columns and the first 32 numerator columns: one wait
+            float v[32], zh, zl;
+            ptx::tmem_ld_32_2cols(taddr, taddr + D, v, zh, zl);
             // NVFP4: phi(q) carries the global scale gq (numerator and denominator alike)
             const float gq = FP4 ? g.gq : 1.0f;
             const float inv = FP4 ? __frcp_rn(gq * zh + gq * zl + g.eps) : __frcp_rn(zh + zl + g.eps);
             uint32_t ow[D / 2];
 #pragma unroll
             for (int half = 0; half < D / 32; ++half) {
-                float v[32];
-                ptx::tmem_ld_32cols(taddr + 32 * half, v);
+                if (half > 0) ptx::tmem_ld_32cols(taddr + 32 * half, v);
                 if constexpr (FP4) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q) v[q] *= gq;
@@ -1112,12 +1112,22 @@ struct Pass2 {
             __nv_bfloat16 *obase = o + (size_t)bb * g.lo.batch + (size_t)hh * g.lo.head;
             store_row<D>(stg, lane, ow);
             __syncwarp();
+            if (g.lo.tok == D) {  // rows contiguous: the warp's 32 rows are one span
+                uint4 *dst = reinterpret_cast<uint4 *>(obase + (size_t)(n + 32 * sub) * D);
 #pragma unroll
-            for (int i = lane; i < 32 * CPR; i += 32) {
-                const int row = i / CPR, jj = i - row * CPR, nr = 32 * sub + row;
-                if (nr < valid)
-                    __stcs(reinterpret_cast<uint4 *>(obase + (size_t)(n + nr) * g.lo.tok) + jj,
-                           *reinterpret_cast<const uint4 *>(stg + swz_chunk<D>(row, jj)));
+                for (int i = lane; i < 32 * CPR; i += 32) {
+                    const int row = i / CPR, jj = i - row * CPR;
+                    if (32 * sub + row < valid)
+                        __stcs(dst + i, *reinterpret_cast<const uint4 *>(stg + swz_chunk<D>(row, jj)));
+                }
+            } else {
+#pragma unroll
+                for (int i = lane; i < 32 * CPR; i += 32) {
+                    const int row = i / CPR, jj = i - row * CPR, nr = 32 * sub + row;
+                    if (nr < valid)
+                        __stcs(reinterpret_cast<uint4 *>(obase + (size_t)(n + nr) * g.lo.tok) + jj,
+                               *reinterpret_cast<const uint4 *>(stg + swz_chunk<D>(row, jj)));
+                }
             }
             __syncwarp();  // the staging is read before the next tile's rows go in
         }

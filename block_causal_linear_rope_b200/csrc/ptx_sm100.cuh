@@ -45,14 +45,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a warp whose phase is not complete sleeps
+// in the barrier unit until the phase completes or about `hint_ns` pass, instead
+// of taking issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 10000000u;  // 10 ms; a completed phase wakes the warp at once
+
 // Bounded wait on an mbarrier phase.  Returns false (and records `code` in
 // *watchdog, first writer wins) if the phase does not complete within
-// limit_ns; the caller then abandons its work instead of hanging.
+// limit_ns; the caller then abandons its work instead of hanging.  The clock
+// is read only when a suspended try_wait gives up, not once per poll.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int *watchdog,
                                                   int code, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t start = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) {
         if (globaltimer_ns() - start > limit_ns) {
             atomicCAS(watchdog, 0, code);
             return false;
@@ -229,6 +247,31 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float (&v)[32]) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 fp32 columns at `taddr` and 2 more at `taddr2` of this thread's TMEM lane,
+// one wait for both loads.
+__device__ __forceinline__ void tmem_ld_32_2cols(uint32_t taddr, uint32_t taddr2, float (&v)[32], float &a,
+                                                 float &b) {
+    uint32_t r[34];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%34];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%32, %33}, [%35];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33])
+        : "r"(taddr), "r"(taddr2)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    a = __uint_as_float(r[32]);
+    b = __uint_as_float(r[33]);
 }
 
 // Shared-memory matrix descriptor (tcgen05 format, version 1).
