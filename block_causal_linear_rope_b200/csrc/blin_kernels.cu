@@ -147,8 +147,8 @@ static cudaError_t launch_ex(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3
 cudaError_t launch_scan(const KGeom &g, int d, const float *S_in, const float *z_in, float *S_out,
                         float *z_out, cudaStream_t s) {
     const long long cols = (long long)g.BH * ((d * d + d) / 4);  // (head, float4 column) pairs: one thread each
-    const dim3 grid((unsigned)((cols + 255) / 256));
-    cudaError_t e = launch_ex(true, scan_kernel, grid, dim3(256), 0, s, g, d, S_in, z_in, S_out, z_out);
+    const dim3 grid((unsigned)((cols + kScanThreads - 1) / kScanThreads));
+    cudaError_t e = launch_ex(true, scan_kernel, grid, dim3(kScanThreads), 0, s, g, d, S_in, z_in, S_out, z_out);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -53,19 +53,20 @@ __global__ void rope_table_kernel(float2 *tab, int T, int t0, int Hg, int Wg, in
 // The order depends only on the block's own length, so a block-by-block
 // stream reproduces a one-shot prefill bit for bit.  (Talk transcript: the
 // new state is the cached state plus the block's contribution.)
-// One thread per (head, float4 column), all heads' columns laid end to end, so
-// the launch is one wave whatever the block count.
-constexpr int kScanLoads = 16;  // chunk partial loads in flight per thread
+// One thread per (head, float4 column), all heads' columns laid end to end, in
+// 128-thread CTAs so that every SM takes a share.
+constexpr int kScanLoads = 8;  // chunk partial loads in flight per thread (a block's chunks, in groups)
+constexpr int kScanThreads = 128;
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
-// Each thread walks its column's (block, chunk) sequence in order, keeping
-// kScanLoads loads in flight across block boundaries; consecutive threads read
-// consecutive columns.
-__global__ void __launch_bounds__(256) scan_kernel(KGeom g, int d, const float *S_in, const float *z_in,
-                                                   float *S_out, float *z_out) {
+// Each thread walks its column block by block: a block's chunk partials are loaded
+// together (up to kScanLoads at a time) and summed in chunk order, then added to the
+// running state.
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(KGeom g, int d, const float *S_in, const float *z_in,
+                                                             float *S_out, float *z_out) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");  // chunk partials come from the previous kernel
     const int E4 = (d * d + d) / 4;
@@ -74,39 +75,25 @@ __global__ void __launch_bounds__(256) scan_kernel(KGeom g, int d, const float *
     const int bh = (int)(f / E4), e4 = (int)(f - (long long)bh * E4);
     const float4 *part = reinterpret_cast<const float4 *>(g.part) + (size_t)bh * g.nblk * g.cpb * E4 + e4;
     float4 *prefix = reinterpret_cast<float4 *>(g.prefix) + (size_t)bh * g.nblk * E4 + e4;
-    auto nchunks = [&](int b) { return units_of_block(g, b, g.nc_first, g.nc_mid, g.nc_last); };
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (S_in != nullptr)
         acc = 4 * e4 < d * d ? reinterpret_cast<const float4 *>(S_in + (size_t)bh * d * d)[e4]
                              : reinterpret_cast<const float4 *>(z_in + (size_t)bh * d)[e4 - d * d / 4];
-    // issue cursor (ib, ic) and consume cursor (cb, cc) over the (block, chunk) sequence
-    int ib = 0, ic = 0, in = g.nblk > 0 ? nchunks(0) : 0;
-    int cb = 0, cc = 0, cn = in;
-    float4 pb = make_float4(0.f, 0.f, 0.f, 0.f);
-    while (cb < g.nblk) {
-        float4 v[kScanLoads];
+    for (int b = 0; b < g.nblk; ++b) {
+        const int nc = units_of_block(g, b, g.nc_first, g.nc_mid, g.nc_last);
+        const float4 *src = part + (size_t)b * g.cpb * E4;
+        float4 pb = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c0 = 0; c0 < nc; c0 += kScanLoads) {
+            float4 v[kScanLoads];
 #pragma unroll
-        for (int j = 0; j < kScanLoads; ++j) {
-            if (ib < g.nblk) {
-                v[j] = __ldcg(part + ((size_t)ib * g.cpb + ic) * E4);
-                if (++ic == in) {
-                    ic = 0;
-                    if (++ib < g.nblk) in = nchunks(ib);
-                }
-            }
-        }
+            for (int j = 0; j < kScanLoads; ++j)
+                if (c0 + j < nc) v[j] = __ldcg(src + (size_t)(c0 + j) * E4);
 #pragma unroll
-        for (int j = 0; j < kScanLoads; ++j) {
-            if (cb < g.nblk) {
-                pb = cc == 0 ? v[j] : f4add(pb, v[j]);
-                if (++cc == cn) {  // block cb complete
-                    acc = f4add(acc, pb);
-                    prefix[(size_t)cb * E4] = acc;
-                    cc = 0;
-                    if (++cb < g.nblk) cn = nchunks(cb);
-                }
-            }
+            for (int j = 0; j < kScanLoads; ++j)
+                if (c0 + j < nc) pb = c0 + j == 0 ? v[j] : f4add(pb, v[j]);
         }
+        acc = f4add(acc, pb);  // block b complete
+        prefix[(size_t)b * E4] = acc;
     }
     if (S_out != nullptr) {
         if (4 * e4 < d * d)
