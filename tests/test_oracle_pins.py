@@ -269,6 +269,39 @@ def test_scale_of_value_is_linear_and_eps_small_limit():
     np.testing.assert_allclose(ones[live], 1.0, rtol=1e-12)
 
 
+def test_positive_scaling_of_q_and_k_cancels_without_eps():
+    """phi is positively homogeneous and o = num / den: with eps = 0, doubling q or k (exact in
+    binary floating point) leaves every output bit unchanged.  A missing normalisation, phi
+    applied after RoPE, or eps inside the dot product would break it."""
+    q, k, v, pos, blk = _small_case(seed=60)
+    rows = np.arange(q.shape[1])
+    base = oracle.attention_rows(q, k, v, pos, blk, rows, (8, 12, 12), 1e4, 0.0)
+    live = np.maximum(q, 0).sum(-1) > 0  # rows whose phi(q) is zero are 0 / 0 without eps
+    for q2, k2 in ((2 * q, k), (q, 2 * k), (0.5 * q, 4 * k)):
+        out = oracle.attention_rows(q2, k2, v, pos, blk, rows, (8, 12, 12), 1e4, 0.0)
+        np.testing.assert_array_equal(out[live], base[live])
+
+
+def test_keys_without_a_positive_feature_contribute_nothing():
+    """A key whose features are all negative has phi(k) = 0, so it adds nothing to S or z: its
+    value rows may be anything.  Using k instead of phi(k) in the numerator or the denominator
+    would make them matter."""
+    q, k, v, pos, blk = _small_case(seed=70)
+    rng = np.random.default_rng(71)
+    dead = rng.random(k.shape[1]) < 0.3
+    k = k.copy()
+    k[:, dead] = -np.abs(k[:, dead])
+    v2 = v.copy()
+    v2[:, dead] = _rand(v2[:, dead].shape, 72, scale=100.0)
+    rows = np.arange(q.shape[1])
+    a = oracle.attention_rows(q, k, v, pos, blk, rows, (8, 12, 12), 1e4, 1e-6)
+    b = oracle.attention_rows(q, k, v2, pos, blk, rows, (8, 12, 12), 1e4, 1e-6)
+    np.testing.assert_array_equal(a, b)
+    s1, _, _ = oracle.recurrence(q, k, v, pos, blk, (8, 12, 12), 1e4, 1e-6)
+    s2, _, _ = oracle.recurrence(q, k, v2, pos, blk, (8, 12, 12), 1e4, 1e-6)
+    np.testing.assert_array_equal(s1, s2)
+
+
 def test_golden_fixture_unchanged():
     """The oracle still produces the recorded tiny-workload rows bit for bit."""
     import json
