@@ -180,3 +180,78 @@ def test_strided_layout_checks(lq, lo, B, code):
         assert rc not in (SHAPE, ALIGN, INVALID), blin.lib.blin_last_error().decode()
     else:
         assert rc == code, blin.lib.blin_last_error().decode()
+
+
+def fp4(data=FAKE, scale=FAKE, gs=1.0):
+    return blin.Nvfp4(data, scale, gs)
+
+
+def prefill_fp4_raw(q=None, k=None, v=None, split=(8, 12, 12)):
+    g = geom(T=4, Hg=4, Wg=4, split=split)
+    q, k, v = q or fp4(), k or fp4(), v or fp4()
+    return blin.lib.blin_prefill_nvfp4(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), FAKE, 1, 2, 32,
+                                       ctypes.byref(g), None, FAKE, 1 << 30, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=fp4(data=None)), INVALID), (dict(k=fp4(scale=None)), INVALID),
+    (dict(v=fp4(data=FAKE + 8)), ALIGN), (dict(q=fp4(scale=FAKE + 4)), ALIGN),
+    (dict(k=fp4(gs=0.0)), INVALID), (dict(v=fp4(gs=-1.0)), INVALID),
+    (dict(q=fp4(gs=float("inf"))), INVALID), (dict(k=fp4(gs=float("nan"))), INVALID),
+    (dict(split=(16, 8, 8)), SHAPE),  # a valid split, but only (8, 12, 12) at d = 32 runs on the tensor cores
+])
+def test_nvfp4_operand_checks(kw, code):
+    assert prefill_fp4_raw(**kw) == code, blin.lib.blin_last_error().decode()
+    assert blin.lib.blin_last_error().decode() != ""
+
+
+def test_nvfp4_null_operand_and_block_step_checks():
+    g = geom(T=3, Hg=4, Wg=4)
+    a = fp4()
+    assert blin.lib.blin_prefill_nvfp4(None, ctypes.byref(a), ctypes.byref(a), FAKE, 1, 2, 32, ctypes.byref(g),
+                                       None, FAKE, 1 << 30, None) == INVALID
+    bad = fp4(gs=0.0)
+    assert blin.lib.blin_block_step_nvfp4(ctypes.byref(a), ctypes.byref(bad), ctypes.byref(a), FAKE, 1, 2, 32,
+                                          ctypes.byref(g), FAKE, 1, None) == INVALID
+    # operands pass, then the state is checked: NULL is refused before any launch
+    assert blin.lib.blin_block_step_nvfp4(ctypes.byref(a), ctypes.byref(a), ctypes.byref(a), FAKE, 1, 2, 32,
+                                          ctypes.byref(g), None, 1, None) == INVALID
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 16, 4, 4, 1), INVALID), ((1, 12, 4, 4, 1), SHAPE), ((1, 16, 0, 4, 1), INVALID), ((1, 16, 4, 4, 7), DTYPE),
+])
+def test_tconv_state_init_checks(args, code):
+    out = ctypes.c_void_p()
+    assert blin.lib.blin_tconv_state_init(*args, None, ctypes.byref(out)) == code
+    assert not out.value
+    assert blin.lib.blin_tconv_state_init(1, 16, 4, 4, 1, None, None) == INVALID  # nowhere to put the handle
+
+
+def test_tconv_state_accessors_reject_null():
+    assert blin.lib.blin_tconv_state_free(None) == OK
+    assert blin.lib.blin_tconv_state_bytes(None) == 0
+    assert blin.lib.blin_tconv_state_frame(None, None, None) == INVALID
+
+
+def tconv_raw(x=FAKE, taps=FAKE, bias=None, y=FAKE, dt=1, B=1, C=16, g=None, st=None, commit=0):
+    g = g if g is not None else geom(T=4, Hg=4, Wg=4)
+    return blin.lib.blin_tconv(x, taps, bias, y, dt, B, C, ctypes.byref(g), st, commit, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), INVALID), (dict(taps=None), INVALID), (dict(y=None), INVALID), (dict(dt=9), DTYPE),
+    (dict(B=0), INVALID), (dict(C=20), SHAPE), (dict(commit=2), INVALID), (dict(commit=1), INVALID),
+    (dict(x=FAKE + 8), ALIGN), (dict(y=FAKE + 2), ALIGN), (dict(taps=FAKE + 2), ALIGN), (dict(bias=FAKE + 1), ALIGN),
+    (dict(g=geom(T=-1, Hg=4, Wg=4)), INVALID), (dict(g=geom(T=4, Hg=0, Wg=4)), INVALID),
+    (dict(g=geom(T=4, Hg=4, Wg=4, F=0)), INVALID),
+])
+def test_tconv_rejects_bad_arguments_before_launch(kw, code):
+    assert tconv_raw(**kw) == code, blin.lib.blin_last_error().decode()
+    assert blin.lib.blin_last_error().decode() != ""
+
+
+def test_tconv_geom_null_and_empty_call():
+    assert blin.lib.blin_tconv(FAKE, FAKE, None, FAKE, 1, 1, 16, None, None, 0, None) == INVALID
+    # no frames and no state: nothing to do, nothing launched
+    assert tconv_raw(g=geom(T=0, Hg=4, Wg=4)) == OK
