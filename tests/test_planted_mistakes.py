@@ -109,7 +109,8 @@ def outcomes(tmp_path_factory):
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", lib, str(c_file),
                                "-lm"])
         libs[name] = (lib, first)
-    with ThreadPoolExecutor(max_workers=max(2, min(len(libs), os.cpu_count() or 2))) as ex:
+    workers = max(2, min(8, len(os.sched_getaffinity(0))))  # each child imports torch: keep the count modest
+    with ThreadPoolExecutor(max_workers=workers) as ex:
         futs = {name: ex.submit(_run_pins, lib, first) for name, (lib, first) in libs.items()}
         return {name: f.result() for name, f in futs.items()}
 
