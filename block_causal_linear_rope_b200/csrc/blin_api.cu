@@ -180,6 +180,25 @@ static Plan make_plan(int B, int H, int d, int T, int Hg, int Wg, int F, int t0,
     return p;
 }
 
+// Launch-shape limits of a plan.  The tensor-core kernels hand out the call's
+// (head, chunk) and (head, query group) units through 32-bit counters that run a
+// few claims past the end; the CUDA-core kernels put blocks and heads on grid y
+// and z, which hold at most 65535 each.
+static constexpr long long kMaxUnits = (1LL << 31) - (1LL << 20);
+static blin_status check_launch_limits(const Plan &p) {
+    const KGeom &g = p.g;
+    if (p.tc) {
+        const long long u1 = (long long)g.BH * g.U1, u2 = (long long)g.BH * g.U2;
+        if (u1 > kMaxUnits || u2 > kMaxUnits)
+            return fail(BLIN_ERR_SHAPE, "too many work units for one call (%lld state chunks, %lld query groups); "
+                                        "split the call over heads or frames", u1, u2);
+    } else if (g.BH > 65535 || g.nblk > 65535) {
+        return fail(BLIN_ERR_SHAPE, "the CUDA-core path takes at most 65535 heads (B*H = %d) and 65535 blocks "
+                                    "(%d) per call; split the call", g.BH, g.nblk);
+    }
+    return BLIN_OK;
+}
+
 // 256 bytes of alignment slack, then the work counters, RoPE table, chunk partials, prefixes
 static size_t plan_bytes(const Plan &p) { return 256 + p.ctl_bytes + p.tab_bytes + p.part_bytes + p.prefix_bytes; }
 
@@ -597,17 +616,19 @@ static blin_status prefill_impl(const void *q, const void *k, const void *v, voi
                         st->d, B, H, d);
     }
     if (g->T == 0) return BLIN_OK;
-    const size_t need = prefill_bytes(B, H, d, g);
-    if (workspace == nullptr || ws_bytes < need)
-        return fail(BLIN_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? ws_bytes : 0, need);
-    if (!aligned16(workspace)) return fail(BLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
     const int t0 = st ? st->t_next : 0;
     if ((long long)t0 + g->T >= (1LL << 30)) return fail(BLIN_ERR_SHAPE, "frame index overflow");
     const bool tc = dt == BLIN_BF16 && tc_supported(d, g->rope_split);
     Plan p = make_plan(B, H, d, g->T, g->Hgt, g->Wid, g->block_frames, t0, false, g->rope_split, g->eps, tc);
+    if ((rc = check_launch_limits(p)) != BLIN_OK) return rc;
     if (fp4 && !p.tc)
         return fail(BLIN_ERR_SHAPE, "NVFP4 inputs need the tensor-core path (rope split (8,12,12) at d=32 or "
                                     "(16,24,24) at d=64, and a RoPE table that fits shared memory)");
+    // the workspace is checked last: every shape and layout check above needs none
+    const size_t need = prefill_bytes(B, H, d, g);
+    if (workspace == nullptr || ws_bytes < need)
+        return fail(BLIN_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? ws_bytes : 0, need);
+    if (!aligned16(workspace)) return fail(BLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
     p.g.lq = lq;
     p.g.lo = lo;
     plan_bind(p, workspace);
@@ -650,6 +671,7 @@ static blin_status block_step_impl(const void *q, const void *k, const void *v, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool tc = dt == BLIN_BF16 && tc_supported(d, g->rope_split);
     Plan p = make_plan(B, H, d, frames, g->Hgt, g->Wid, frames, st->t_next, true, g->rope_split, g->eps, tc);
+    if ((rc = check_launch_limits(p)) != BLIN_OK) return rc;
     if (fp4 && !p.tc)
         return fail(BLIN_ERR_SHAPE, "NVFP4 inputs need the tensor-core path (rope split (8,12,12) at d=32 or "
                                     "(16,24,24) at d=64, and a RoPE table that fits shared memory)");

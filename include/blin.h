@@ -159,7 +159,11 @@ BLIN_API size_t blin_prefill_workspace_size(int B, int H, int d, const blin_geom
  * at block boundaries gives the same rows as one call, and the final (S, z) is
  * bitwise equal to the one blin_block_step reaches over the same blocks.  A
  * call that ends inside a block lets that block's rows see only the frames
- * given so far; the next call's rows of the same block see the whole block. */
+ * given so far; the next call's rows of the same block see the whole block.
+ * Per-call limits (BLIN_ERR_SHAPE beyond them, before any launch): on the
+ * tensor-core path fewer than 2^31 - 2^20 (head, state chunk) and (head, query
+ * group) work units; on the CUDA-core path at most 65535 heads (B*H) and 65535
+ * causal blocks.  Larger jobs split over heads or frames. */
 BLIN_API blin_status blin_prefill(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                          int B, int H, int d, const blin_geom *g, blin_state *st,
                          void *workspace, size_t ws_bytes, blin_stream stream);
@@ -196,7 +200,8 @@ BLIN_API blin_status blin_prefill_strided(const void *q, const void *k, const vo
  * blin_prefill does, so a block-by-block stream gives bitwise the outputs and
  * the final (S, z) of one prefill over the same frames.  Needs scratch owned
  * by the state; the first call with a larger block grows it (allocation on
- * stream), blin_state_reserve avoids that. */
+ * stream), blin_state_reserve avoids that.  Per-call limits as for
+ * blin_prefill. */
 BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                             int B, int H, int d, const blin_geom *g, blin_state *st, int commit,
                             blin_stream stream);

@@ -1,7 +1,10 @@
 """C-ABI checks that need no GPU: symbols, sizes and host-side argument validation.
 
-Every call here returns before any CUDA launch (the checks run first), so the
-library can be exercised on a machine without a device.
+Every call here is refused by a host check before any device work: calls
+meant to pass the shape and layout checks give no workspace, and the workspace
+check is the last one before the library touches a device.  So the library is
+exercised on a machine without a device, and these calls stay on the host on a
+machine with one (the addresses passed are never dereferenced).
 """
 import ctypes
 import os
@@ -162,8 +165,10 @@ def test_version_string():
 def strided_raw(lq=None, lo=None, dt=1, d=32, H=2, B=1):
     g = geom(T=4, Hg=4, Wg=4)
     mk = lambda t: None if t is None else ctypes.byref(blin.Layout(*t))
+    # no workspace: a call whose layouts pass stops at the workspace check, the last
+    # one before any device work, so these calls never touch a device
     return blin.lib.blin_prefill_strided(FAKE, FAKE, FAKE, FAKE, dt, B, H, d, ctypes.byref(g), mk(lq), mk(lo), None,
-                                         FAKE, 1 << 30, None)
+                                         None, 0, None)
 
 
 @pytest.mark.parametrize("lq,lo,B,code", [
@@ -176,8 +181,8 @@ def strided_raw(lq=None, lo=None, dt=1, d=32, H=2, B=1):
 def test_strided_layout_checks(lq, lo, B, code):
     rc = strided_raw(lq=lq, lo=lo, B=B)
     if code == OK:
-        # valid layouts pass every host check and only then reach the (absent) device
-        assert rc not in (SHAPE, ALIGN, INVALID), blin.lib.blin_last_error().decode()
+        # valid layouts pass every shape and layout check
+        assert rc == WORKSPACE, blin.lib.blin_last_error().decode()
     else:
         assert rc == code, blin.lib.blin_last_error().decode()
 
@@ -190,7 +195,7 @@ def prefill_fp4_raw(q=None, k=None, v=None, split=(8, 12, 12)):
     g = geom(T=4, Hg=4, Wg=4, split=split)
     q, k, v = q or fp4(), k or fp4(), v or fp4()
     return blin.lib.blin_prefill_nvfp4(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), FAKE, 1, 2, 32,
-                                       ctypes.byref(g), None, FAKE, 1 << 30, None)
+                                       ctypes.byref(g), None, None, 0, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -209,7 +214,10 @@ def test_nvfp4_null_operand_and_block_step_checks():
     g = geom(T=3, Hg=4, Wg=4)
     a = fp4()
     assert blin.lib.blin_prefill_nvfp4(None, ctypes.byref(a), ctypes.byref(a), FAKE, 1, 2, 32, ctypes.byref(g),
-                                       None, FAKE, 1 << 30, None) == INVALID
+                                       None, None, 0, None) == INVALID
+    # valid operands on the tensor-core split stop at the missing workspace
+    assert blin.lib.blin_prefill_nvfp4(ctypes.byref(a), ctypes.byref(a), ctypes.byref(a), FAKE, 1, 2, 32,
+                                       ctypes.byref(g), None, None, 0, None) == WORKSPACE
     bad = fp4(gs=0.0)
     assert blin.lib.blin_block_step_nvfp4(ctypes.byref(a), ctypes.byref(bad), ctypes.byref(a), FAKE, 1, 2, 32,
                                           ctypes.byref(g), FAKE, 1, None) == INVALID
@@ -255,3 +263,23 @@ def test_tconv_geom_null_and_empty_call():
     assert blin.lib.blin_tconv(FAKE, FAKE, None, FAKE, 1, 1, 16, None, None, 0, None) == INVALID
     # no frames and no state: nothing to do, nothing launched
     assert tconv_raw(g=geom(T=0, Hg=4, Wg=4)) == OK
+
+
+@pytest.mark.parametrize("dt,H,T,F,msg", [
+    (1, 1 << 22, 512, 1, "work units"),      # tensor-core path: 2^31 (head, chunk) units
+    (0, 70000, 1, 1, "65535 heads"),         # CUDA-core path: heads on grid z
+    (0, 2, 70000, 1, "65535 heads"),         # CUDA-core path: blocks on grid y (same message)
+])
+def test_launch_limits_are_refused_before_launch(dt, H, T, F, msg):
+    g = geom(T=T, Hg=1, Wg=1, F=F)
+    rc = blin.lib.blin_prefill(FAKE, FAKE, FAKE, FAKE, dt, 1, H, 32, ctypes.byref(g), None, None, 0, None)
+    assert rc == SHAPE
+    assert msg in blin.lib.blin_last_error().decode()
+
+
+@pytest.mark.parametrize("dt,H,T", [(1, (1 << 22) - 4096, 512), (0, 65535, 1), (0, 2, 65535)])
+def test_just_inside_the_launch_limits(dt, H, T):
+    # passes the shape checks and stops at the (missing) workspace, before any device work
+    g = geom(T=T, Hg=1, Wg=1, F=1)
+    rc = blin.lib.blin_prefill(FAKE, FAKE, FAKE, FAKE, dt, 1, H, 32, ctypes.byref(g), None, None, 0, None)
+    assert rc == WORKSPACE, blin.lib.blin_last_error().decode()
