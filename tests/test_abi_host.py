@@ -283,3 +283,40 @@ def test_just_inside_the_launch_limits(dt, H, T):
     g = geom(T=T, Hg=1, Wg=1, F=1)
     rc = blin.lib.blin_prefill(FAKE, FAKE, FAKE, FAKE, dt, 1, H, 32, ctypes.byref(g), None, None, 0, None)
     assert rc == WORKSPACE, blin.lib.blin_last_error().decode()
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "blin.h"
+
+int main(void) {
+    blin_geom g;
+    memset(&g, 0, sizeof g);
+    g.T = 21; g.Hgt = 45; g.Wid = 80; g.block_frames = 3;
+    g.rope_split[0] = 8; g.rope_split[1] = 12; g.rope_split[2] = 12;
+    g.theta = 10000.0f; g.eps = 1e-6f;
+    size_t ws = blin_prefill_workspace_size(1, 70, 32, &g);
+    blin_status rc = blin_prefill(NULL, NULL, NULL, NULL, BLIN_BF16, 1, 70, 32, &g, NULL, NULL, 0, NULL);
+    printf("%s|%zu|%d|%s\n", blin_version(), ws, (int)rc, blin_last_error());
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_builds_links_and_calls(tmp_path):
+    """The boundary is usable from C99 alone: header, shared library, no Python or torch types."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = str(tmp_path / "client")
+    pkg = os.path.dirname(blin.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-o", exe, "-L", pkg, "-lblin", "-Wl,-rpath," + pkg])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120, check=True).stdout.strip()
+    version, ws_c, rc, msg = out.split("|", 3)
+    assert version == blin.lib.blin_version().decode()
+    assert int(ws_c) == ws(1, 70, 32, geom(T=21, Hg=45, Wg=80))
+    assert int(rc) == INVALID and msg
+    # and the header is valid C++ as well
+    subprocess.check_call(["g++", "-std=c++11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-x",
+                           "c++", HEADER])
