@@ -216,6 +216,34 @@ def _check_qkv(q, k, v):
         raise ValueError("q, k and v must share shape and dtype")
     if not (q.stride() == k.stride() == v.stride()):
         raise ValueError("q, k and v must share strides (one layout for the three)")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k and v must be on one device")
+    _check_device(q)
+
+
+def _check_device(t: torch.Tensor) -> None:
+    """The library launches on the current device: the call's tensors must live there."""
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {t.device} but the current device is cuda:{torch.cuda.current_device()}; "
+                         "call under torch.cuda.device(...)")
+
+
+def _check_out(out, shape, dtype, device, contiguous: bool = False) -> None:
+    """A caller-given output must match the call (the library cannot see its extent)."""
+    if (not isinstance(out, torch.Tensor) or out.device != device or out.dtype != dtype
+            or tuple(out.shape) != tuple(shape) or out.stride(-1) != 1 or (contiguous and not out.is_contiguous())):
+        what = "contiguous " if contiguous else ""
+        raise ValueError(f"out must be a {what}{dtype} tensor of shape {tuple(shape)} on {device}, last dimension "
+                         "contiguous")
+
+
+def _workspace_arg(workspace, need: int, device):
+    """(pointer, bytes) of a caller-given workspace, or of a new one of `need` bytes."""
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    elif not isinstance(workspace, torch.Tensor) or workspace.device != device or not workspace.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    return workspace, ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
 
 
 def _layouts(q: torch.Tensor, out: torch.Tensor):
@@ -253,13 +281,13 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Sequence[in
     g = _geom(T, Hg, Wg, block_frames, rope_split, theta, eps)
     if out is None:
         out = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
+    else:
+        _check_out(out, (B, H, N, d), q.dtype, q.device)
     need = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    workspace, ws_ptr, ws_bytes = _workspace_arg(workspace, need, q.device)
     args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
             ctypes.c_void_p(out.data_ptr()), _dtype_code(q), B, H, d, ctypes.byref(g))
-    tail = (state.handle if state is not None else None, ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
-            _stream(stream))
+    tail = (state.handle if state is not None else None, ws_ptr, ws_bytes, _stream(stream))
     lays = _layouts(q, out)
     if lays is None:
         _check(lib.blin_prefill(*args, *tail))
@@ -282,6 +310,8 @@ def block_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Hg: int, Wg: i
         raise ValueError(f"N={N} but frames*Hg*Wg={frames * Hg * Wg}")
     if out is None:
         out = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
+    else:
+        _check_out(out, (B, H, N, d), q.dtype, q.device)
     g = _geom(frames, Hg, Wg, frames if block_frames is None else block_frames, rope_split, theta, eps)
     args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
             ctypes.c_void_p(out.data_ptr()), _dtype_code(q), B, H, d, ctypes.byref(g))
@@ -435,11 +465,16 @@ def tconv(x: torch.Tensor, taps: torch.Tensor, bias: Optional[torch.Tensor], gri
     T, Hg, Wg = (int(v) for v in grid)
     if N != T * Hg * Wg:
         raise ValueError(f"N={N} but T*Hg*Wg={T * Hg * Wg}")
+    _check_device(x)
+    if taps.numel() != 3 * C or (bias is not None and bias.numel() != C):
+        raise ValueError(f"taps must hold [C, 3] = {3 * C} values and bias [C] = {C}")
     taps = taps.to(device=x.device, dtype=torch.float32).contiguous()
     if bias is not None:
         bias = bias.to(device=x.device, dtype=torch.float32).contiguous()
     if out is None:
         out = torch.empty_like(x)
+    else:
+        _check_out(out, x.shape, x.dtype, x.device, contiguous=True)
     g = _geom(T, Hg, Wg, block_frames, (0, 0, 0), 1e4, 0.0)
     _check(lib.blin_tconv(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(taps.data_ptr()),
                           None if bias is None else ctypes.c_void_p(bias.data_ptr()), ctypes.c_void_p(out.data_ptr()),
@@ -474,6 +509,14 @@ class Nvfp4Tensor:
         return Nvfp4(ctypes.c_void_p(self.data.data_ptr()), ctypes.c_void_p(self.scale.data_ptr()), self.global_scale)
 
 
+def _nvfp4_device(q: "Nvfp4Tensor", k: "Nvfp4Tensor", v: "Nvfp4Tensor") -> torch.device:
+    dev = q.data.device
+    if not all(t.data.device == dev and t.scale.device == dev for t in (q, k, v)):
+        raise ValueError("q, k and v must be on one device")
+    _check_device(q.data)
+    return dev
+
+
 def prefill_nvfp4(q: Nvfp4Tensor, k: Nvfp4Tensor, v: Nvfp4Tensor, grid: Sequence[int], block_frames: int,
                   rope_split: Sequence[int], theta: float = 1e4, eps: float = 1e-6,
                   state: Optional[BlockState] = None, out: Optional[torch.Tensor] = None,
@@ -486,15 +529,17 @@ def prefill_nvfp4(q: Nvfp4Tensor, k: Nvfp4Tensor, v: Nvfp4Tensor, grid: Sequence
     if N != T * Hg * Wg:
         raise ValueError(f"N={N} but T*Hg*Wg={T * Hg * Wg}")
     g = _geom(T, Hg, Wg, block_frames, rope_split, theta, eps)
+    dev = _nvfp4_device(q, k, v)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.data.device)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_out(out, (B, H, N, d), torch.bfloat16, dev, contiguous=True)
     need = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.data.device)
+    workspace, ws_ptr, ws_bytes = _workspace_arg(workspace, need, dev)
     qc, kc, vc = q.c(), k.c(), v.c()
     _check(lib.blin_prefill_nvfp4(ctypes.byref(qc), ctypes.byref(kc), ctypes.byref(vc), ctypes.c_void_p(out.data_ptr()),
                                   B, H, d, ctypes.byref(g), state.handle if state is not None else None,
-                                  ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)))
+                                  ws_ptr, ws_bytes, _stream(stream)))
     return out
 
 
@@ -503,11 +548,16 @@ def block_step_nvfp4(q: Nvfp4Tensor, k: Nvfp4Tensor, v: Nvfp4Tensor, Hg: int, Wg
                      commit: bool = True, out: Optional[torch.Tensor] = None, stream=None,
                      block_frames: Optional[int] = None) -> torch.Tensor:
     """block_step() on NVFP4 q, k, v; the output is bf16."""
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k and v must share a shape")
     B, H, N, d = q.shape
     if N != frames * Hg * Wg:
         raise ValueError(f"N={N} but frames*Hg*Wg={frames * Hg * Wg}")
+    dev = _nvfp4_device(q, k, v)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.data.device)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_out(out, (B, H, N, d), torch.bfloat16, dev, contiguous=True)
     g = _geom(frames, Hg, Wg, frames if block_frames is None else block_frames, rope_split, theta, eps)
     qc, kc, vc = q.c(), k.c(), v.c()
     _check(lib.blin_block_step_nvfp4(ctypes.byref(qc), ctypes.byref(kc), ctypes.byref(vc),

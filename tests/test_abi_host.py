@@ -320,3 +320,38 @@ def test_plain_c_client_builds_links_and_calls(tmp_path):
     # and the header is valid C++ as well
     subprocess.check_call(["g++", "-std=c++11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-x",
                            "c++", HEADER])
+
+
+# --------------------------------------------------------------------------- binding-side checks of caller buffers
+def test_binding_checks_a_caller_given_output():
+    import torch
+    cpu = torch.device("cpu")
+    ok = torch.empty(2, 3, 64, 32, dtype=torch.bfloat16)
+    blin._check_out(ok, (2, 3, 64, 32), torch.bfloat16, cpu)
+    blin._check_out(torch.empty(2, 64, 3, 32, dtype=torch.bfloat16).permute(0, 2, 1, 3), (2, 3, 64, 32),
+                    torch.bfloat16, cpu)  # a strided view is fine where layouts are taken
+    for bad in (torch.empty(2, 3, 63, 32, dtype=torch.bfloat16),   # too few rows: the kernels would write past it
+                torch.empty(2, 3, 64, 32, dtype=torch.float32),    # wrong dtype
+                torch.empty(2, 3, 32, 64, dtype=torch.bfloat16).transpose(2, 3),  # d not contiguous
+                "not a tensor"):
+        with pytest.raises(ValueError):
+            blin._check_out(bad, (2, 3, 64, 32), torch.bfloat16, cpu)
+    with pytest.raises(ValueError):  # entry points without layouts want a contiguous output
+        blin._check_out(torch.empty(2, 64, 3, 32, dtype=torch.bfloat16).permute(0, 2, 1, 3), (2, 3, 64, 32),
+                        torch.bfloat16, cpu, contiguous=True)
+    with pytest.raises(ValueError):  # another device
+        blin._check_out(torch.empty(2, 3, 64, 32, dtype=torch.bfloat16, device="meta"), (2, 3, 64, 32),
+                        torch.bfloat16, cpu)
+
+
+def test_binding_passes_workspace_bytes_not_elements():
+    import torch
+    cpu = torch.device("cpu")
+    ws, ptr, nbytes = blin._workspace_arg(None, 1000, cpu)
+    assert nbytes == 1000 and ptr.value == ws.data_ptr()
+    ws, _, nbytes = blin._workspace_arg(torch.empty(300, dtype=torch.float32), 1000, cpu)
+    assert nbytes == 1200
+    with pytest.raises(ValueError):
+        blin._workspace_arg(torch.empty(600, dtype=torch.uint8)[::2], 100, cpu)  # not contiguous
+    with pytest.raises(ValueError):
+        blin._workspace_arg(torch.empty(600, dtype=torch.uint8, device="meta"), 100, cpu)  # another device
