@@ -237,6 +237,21 @@ def _check_out(out, shape, dtype, device, contiguous: bool = False) -> None:
                          "contiguous")
 
 
+def _check_no_overlap(out: torch.Tensor, *inputs: torch.Tensor) -> None:
+    """The output must not overlap an input (the kernels read inputs after writing outputs).
+    Contiguous tensors are compared by address range; strided views, which may interleave
+    without sharing an element, only by start address."""
+    def span(t):
+        return t.data_ptr(), t.data_ptr() + t.numel() * t.element_size()
+    for t in inputs:
+        if out.data_ptr() == t.data_ptr():
+            raise ValueError("out must not overlap the inputs")
+        if out.is_contiguous() and t.is_contiguous():
+            (a0, a1), (b0, b1) = span(out), span(t)
+            if a0 < b1 and b0 < a1:
+                raise ValueError("out must not overlap the inputs")
+
+
 def _workspace_arg(workspace, need: int, device):
     """(pointer, bytes) of a caller-given workspace, or of a new one of `need` bytes."""
     if workspace is None:
@@ -283,6 +298,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Sequence[in
         out = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
     else:
         _check_out(out, (B, H, N, d), q.dtype, q.device)
+        _check_no_overlap(out, q, k, v)
     need = int(lib.blin_prefill_workspace_size(B, H, d, ctypes.byref(g)))
     workspace, ws_ptr, ws_bytes = _workspace_arg(workspace, need, q.device)
     args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
@@ -312,6 +328,7 @@ def block_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Hg: int, Wg: i
         out = torch.empty((B, H, N, d), dtype=q.dtype, device=q.device)
     else:
         _check_out(out, (B, H, N, d), q.dtype, q.device)
+        _check_no_overlap(out, q, k, v)
     g = _geom(frames, Hg, Wg, frames if block_frames is None else block_frames, rope_split, theta, eps)
     args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
             ctypes.c_void_p(out.data_ptr()), _dtype_code(q), B, H, d, ctypes.byref(g))
@@ -475,6 +492,7 @@ def tconv(x: torch.Tensor, taps: torch.Tensor, bias: Optional[torch.Tensor], gri
         out = torch.empty_like(x)
     else:
         _check_out(out, x.shape, x.dtype, x.device, contiguous=True)
+        _check_no_overlap(out, x)
     g = _geom(T, Hg, Wg, block_frames, (0, 0, 0), 1e4, 0.0)
     _check(lib.blin_tconv(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(taps.data_ptr()),
                           None if bias is None else ctypes.c_void_p(bias.data_ptr()), ctypes.c_void_p(out.data_ptr()),

@@ -355,3 +355,18 @@ def test_binding_passes_workspace_bytes_not_elements():
         blin._workspace_arg(torch.empty(600, dtype=torch.uint8)[::2], 100, cpu)  # not contiguous
     with pytest.raises(ValueError):
         blin._workspace_arg(torch.empty(600, dtype=torch.uint8, device="meta"), 100, cpu)  # another device
+
+
+def test_binding_refuses_an_output_over_an_input():
+    import torch
+    buf = torch.empty(2, 3, 64, 32)
+    q = buf[:1]
+    blin._check_no_overlap(buf[1:], q)                      # disjoint halves of one buffer
+    for bad in (buf[:1], buf[0:2].reshape(2, 3, 64, 32)[:1]):
+        with pytest.raises(ValueError):
+            blin._check_no_overlap(bad, q)
+    with pytest.raises(ValueError):
+        blin._check_no_overlap(buf.view(-1)[16:].view(-1)[: 64 * 32].view(1, 1, 64, 32), q)  # shifted, overlapping
+    fused = torch.empty(2, 64, 4, 3, 32)                    # [B, N, 4, H, d]: q, k, v and o interleaved
+    views = [fused[:, :, i].permute(0, 2, 1, 3) for i in range(4)]
+    blin._check_no_overlap(views[3], *views[:3])            # interleaved, no shared element: accepted
