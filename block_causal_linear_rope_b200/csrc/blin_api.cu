@@ -543,8 +543,16 @@ blin_status blin_state_copy_from_host(blin_state *st, const void *host, size_t b
 // Grows the state's block-step scratch to `need` bytes.
 static blin_status ensure_scratch(blin_state *st, size_t need, cudaStream_t s) {
     if (st->scratch_bytes >= need) return BLIN_OK;
+    // Growing inside stream capture would make the state hold graph-owned memory
+    // that later calls outside the graph reuse: refuse, and let the caller reserve.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "stream capture query");
+    if (cap != cudaStreamCaptureStatusNone)
+        return fail(BLIN_ERR_WORKSPACE, "the state's block-step scratch must grow to %zu bytes, which cannot happen "
+                                        "during stream capture: call blin_state_reserve before capturing", need);
     void *p = nullptr;
-    cudaError_t e = cudaMallocAsync(&p, need, s);
+    e = cudaMallocAsync(&p, need, s);
     if (e != cudaSuccess) {
         if (p) cudaFreeAsync(p, s);
         return cuda_fail(e, "block-step scratch allocation");

@@ -200,7 +200,9 @@ BLIN_API blin_status blin_prefill_strided(const void *q, const void *k, const vo
  * blin_prefill does, so a block-by-block stream gives bitwise the outputs and
  * the final (S, z) of one prefill over the same frames.  Needs scratch owned
  * by the state; the first call with a larger block grows it (allocation on
- * stream), blin_state_reserve avoids that.  Per-call limits as for
+ * stream), blin_state_reserve avoids that.  Inside stream capture (a CUDA
+ * graph) the scratch cannot grow: such a call returns BLIN_ERR_WORKSPACE, so
+ * reserve (or run one block step) before capturing.  Per-call limits as for
  * blin_prefill. */
 BLIN_API blin_status blin_block_step(const void *q, const void *k, const void *v, void *o, blin_dtype dt,
                             int B, int H, int d, const blin_geom *g, blin_state *st, int commit,
