@@ -63,10 +63,10 @@ typedef void *blin_stream; /* a cudaStream_t */
 typedef enum {
     BLIN_OK = 0,
     BLIN_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, bad flag, eps/theta out of range */
-    BLIN_ERR_SHAPE = -2,       /* d not 32/64, bad rope split, frames > block_frames, size overflow */
+    BLIN_ERR_SHAPE = -2,       /* d not 32/64, bad rope split, a block step across blocks, size or launch limits */
     BLIN_ERR_DTYPE = -3,       /* unknown dtype */
     BLIN_ERR_ALIGN = -4,       /* q/k/v/o/workspace not 16-byte aligned */
-    BLIN_ERR_WORKSPACE = -5,   /* workspace too small */
+    BLIN_ERR_WORKSPACE = -5,   /* workspace missing or too small; state scratch that would grow during capture */
     BLIN_ERR_STATE = -6,       /* freed/foreign state, B/H/d mismatch, wrong device, wrong byte count */
     BLIN_ERR_CUDA = -7,        /* a CUDA runtime/driver call failed */
     BLIN_ERR_DEVICE = -8       /* a kernel's bounded wait ran out (see blin_device_status) */
