@@ -608,6 +608,7 @@ static blin_status prefill_impl(const void *q, const void *k, const void *v, voi
                                 int d, const blin_geom *g, const blin_layout *lqkv, const blin_layout *lout,
                                 blin_state *st, void *workspace, size_t ws_bytes, blin_stream stream,
                                 const Fp4In *fp4 = nullptr) {
+    const TraceRange trace(fp4 ? "blin_prefill_nvfp4" : (lqkv || lout) ? "blin_prefill_strided" : "blin_prefill");
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;
@@ -654,6 +655,8 @@ static blin_status block_step_impl(const void *q, const void *k, const void *v, 
                                    int H, int d, const blin_geom *g, const blin_layout *lqkv,
                                    const blin_layout *lout, blin_state *st, int commit, blin_stream stream,
                                    const Fp4In *fp4 = nullptr) {
+    const TraceRange trace(fp4 ? "blin_block_step_nvfp4"
+                               : (lqkv || lout) ? "blin_block_step_strided" : "blin_block_step");
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     blin_status rc = check_common(B, H, d, g->T, g->Hgt, g->Wid, g->rope_split, g->theta, g->eps);
     if (rc != BLIN_OK) return rc;

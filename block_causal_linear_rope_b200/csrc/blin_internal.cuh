@@ -5,11 +5,23 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <mutex>
 
 #include "../../include/blin.h"
 
 namespace blin {
+
+// A named NVTX range around one library call, so that profiler timelines group
+// a call's launches under its entry point.  Without an attached tool the push
+// and pop are calls to empty functions.
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange &) = delete;
+    TraceRange &operator=(const TraceRange &) = delete;
+};
 
 // Tokens per TMA tile (and MMA row block).
 constexpr int kTile = 128;

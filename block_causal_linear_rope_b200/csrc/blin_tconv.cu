@@ -252,6 +252,7 @@ size_t blin_tconv_state_bytes(const blin_tconv_state *st) {
 
 blin_status blin_tconv(const void *x, const float *taps, const float *bias, void *y, blin_dtype dt, int B, int C,
                        const blin_geom *g, blin_tconv_state *st, int commit, blin_stream stream) {
+    const blin::TraceRange trace("blin_tconv");
     if (g == nullptr) return fail(BLIN_ERR_INVALID_ARG, "geom is NULL");
     if (x == nullptr || y == nullptr || taps == nullptr)
         return fail(BLIN_ERR_INVALID_ARG, "x, taps and y must be non-NULL device pointers");
