@@ -1,5 +1,5 @@
-// Tensor-core path for bf16 Q/K/V on sm_100a (d = 32 or 64): two persistent
-// warp-specialized kernels around the fixed-order block scan.
+// Tensor-core path for bf16 (or NVFP4) Q/K/V on sm_100a (d = 32 or 64): two
+// persistent warp-specialized kernels around the fixed-order block scan.
 //
 // Pass 1, partial_tc_kernel: per state chunk (whole 128-token tiles of one
 //   block of one head) the partial states P = sum (R_m phi(k_m)) v_m^T and
@@ -15,7 +15,10 @@
 // pipeline is split into roles -- a TMA producer, four transform warps, one
 // MMA-issuing thread, four epilogue warps -- that hand tiles to each other
 // through mbarrier rings, and takes its work units one at a time from a
-// counter shared by the whole grid.  Every wait is bounded.
+// counter shared by the whole grid.  Every wait is bounded.  With NVFP4 inputs
+// the producer lands the packed codes and their block scales, and the
+// transform warps decode them (E2M1 x E4M3 products are exact in bf16) before
+// phi and RoPE; the global scales are applied in fp32.
 #pragma once
 
 #include <cuda_bf16.h>
