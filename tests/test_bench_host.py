@@ -9,6 +9,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 import bench  # noqa: E402
+import workloads  # noqa: E402
 
 
 def test_comment_stripping_keeps_code_and_strings():
@@ -49,3 +50,17 @@ def test_recorded_traffic_requires_matching_hash(tmp_path, monkeypatch):
 @pytest.mark.parametrize("ranks,units,ms,want", [(1, 1000, 1.0, 1e6), (4, 1000, 2.0, 2e6)])
 def test_job_throughput_counts_every_rank(ranks, units, ms, want):
     assert bench.job_throughput(units, ranks, ms) == pytest.approx(want)
+
+
+@pytest.mark.parametrize("name,mb", [("480p", 587.1), ("720p", 1354.8), ("wide", 2147.0), ("decode", 83.9)])
+def test_algorithmic_bytes_per_step_match_the_workload_table(name, mb):
+    """The roofline numerator: Q, K, V read once and O written once per token*head, summed
+    over the launches that move per-token bytes (for decode: one block of 3 frames)."""
+    import block_causal_linear_rope_b200 as blin
+    w = workloads.CONFIGS[name]
+    tokens = w.F * w.HW if name == "decode" else w.N
+    elem = 2 if w.dtype == "bf16" else 4
+    units = w.B * w.H * tokens
+    total = sum(blin.KERNEL_BYTES_PER_UNIT[k] * w.d * elem * units for k in blin.KERNEL_BYTES_PER_UNIT)
+    assert total == units * 4 * w.d * elem
+    assert round(total / 1e6, 1) == mb
