@@ -1,6 +1,6 @@
 """Host-side logic of bench.py that needs no GPU: the source hash that keys
-recorded ncu counters, the reference arm's per-step sample size, and the
-per-rank helpers' arithmetic."""
+recorded ncu counters, the reference arm's per-step sample size, the
+per-rank helpers' arithmetic and the roofline's algorithmic bytes."""
 import os
 import sys
 
